@@ -1,0 +1,323 @@
+"""Benchmark of the grouped-int4 routed-expert FFN layer on B200.
+
+One step = one moe_expert_ffn call (router, on-device row map, fused gate+up+SiLU,
+down projection, weighted scatter-add) over one batch of synthetic input.  Default
+workload: batched decode, 32 tokens, hidden 6144, 256 experts of intermediate 2048,
+top-8, skewed routing (16 hot experts get +3 on logits of variance 2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  N > 1 (under torchrun): independent replicas, one per
+GPU (the layer has no exchange step), weak scaling, time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from weight_only_int4_gq4_b200 import synth  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "weight_only_int4_gq4_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(cfg: synth.MoEConfig, budget_s: float = 12.0, max_tokens: int = 16):
+    """The oracle as it stands, on host cores, over a bounded sample of the workload's
+    tokens (whole MoE layer per token: gate+up+SiLU and down of its K experts)."""
+    import oracle
+    lg, _ = cfg.logits()
+    x = cfg.x()
+    st, idx, wts, _ = oracle.route(lg, cfg.K)
+    order = cfg.sample_tokens() if cfg.oracle_sample else np.arange(cfg.T)
+    experts = {}
+    done, elapsed = 0, 0.0
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    for t in order[:max_tokens]:
+        need = [int(e) for e in idx[t]]
+        for e in need:
+            if e not in experts:
+                experts[e] = (cfg.gate(e), cfg.up(e), cfg.down(e))
+        # a compact stack holding only this token's experts (oracle takes stacked arrays)
+        loc = {e: i for i, e in enumerate(need)}
+        pg = np.stack([experts[e][0][0] for e in need]); sg = np.stack([experts[e][0][1] for e in need])
+        pu = np.stack([experts[e][1][0] for e in need]); su = np.stack([experts[e][1][1] for e in need])
+        pd = np.stack([experts[e][2][0] for e in need]); sd = np.stack([experts[e][2][1] for e in need])
+        idx_l = np.zeros_like(idx)
+        idx_l[t] = [loc[e] for e in need]
+        t0 = time.perf_counter()
+        oracle.moe_tokens(pg, sg, pu, su, pd, sd, cfg.H, cfg.F, x, idx_l, wts, np.array([t]))
+        elapsed += time.perf_counter() - t0
+        done += 1
+        if elapsed >= budget_s:
+            break
+    return {"value": done / elapsed, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} token(s) of {cfg.name}, whole layer per token (K={cfg.K} experts), "
+                      f"{elapsed:.1f} s, fp64 plain C"}
+
+
+def alg_bytes(cfg, n_active):
+    """Algorithmic HBM bytes per step: packed weights + scales of the experts touched,
+    plus activations, logits, h and y traffic."""
+    per_w = lambda O, I: O * (I // 2) + O * (I // 64) * 4  # noqa: E731
+    gate_up = n_active * 2 * per_w(cfg.F, cfg.H)
+    down = n_active * per_w(cfg.H, cfg.F)
+    n = cfg.T * cfg.K
+    x = cfg.T * cfg.H * 2
+    h = n * cfg.F * 2
+    y = cfg.T * cfg.H * 4
+    return {"gate_up": gate_up + x + h, "down": down + h + y * 2, "step": gate_up + down + x + 2 * h + 2 * y
+            + cfg.T * cfg.E * 4}
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    import oracle  # noqa: F401
+    per = []
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(cfg, budget_s=0.0, max_tokens=1)
+        if i >= args.warmup:
+            per.append(1.0 / cb["value"])
+    sec = float(np.mean(per))
+    v = 1.0 / sec
+    line = {"impl": "reference", "metric": "expert-FFN tokens/s (MoE layer, 1 B200)", "value": v,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "F": cfg.F, "K": cfg.K,
+                       "step": "1 sampled token through the CPU oracle"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cb["cores"], "kind": "oracle",
+                             "sample": "1 token per step, whole layer (K experts), fp64 plain C"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=synth.MOE_BATCHED.name, choices=list(synth.MOE_CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = synth.MOE_CONFIGS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    from weight_only_int4_gq4_b200 import gq4
+
+    # ---- inputs resident in HBM (weights of all E experts, logits, x)
+    def stack(fn):
+        parts = [fn(e) for e in range(cfg.E)]
+        return np.stack([a for a, _ in parts]), np.stack([b for _, b in parts])
+
+    Wg = gq4.upload(*stack(cfg.gate))
+    Wu = gq4.upload(*stack(cfg.up))
+    Wd = gq4.upload(*stack(cfg.down))
+    lg_h, _ = cfg.logits()
+    x_h = cfg.x()
+    logits = torch.from_numpy(lg_h).to(dev)
+    x = torch.from_numpy(x_h.view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.empty(cfg.T, cfg.H, dtype=torch.float32, device=dev)
+    ws = gq4.MoEWorkspace(cfg.T, cfg.E, cfg.K, cfg.H, cfg.F, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    n_slots = cfg.T * cfg.K
+    launches_per_step = 3 if n_slots <= 1024 else 6
+
+    def step(ev=None):
+        gq4.moe_expert_ffn(Wg, Wu, Wd, logits, x, cfg.K, y=y, ws=ws, stage_events=ev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n_active = int(ws.routing()["n_active"].cpu()[0])
+    assert ws.status() == 0
+
+    # ---- device-timed steps (L2 flushed between steps, outside the events)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            step(evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)])
+    step_ms = stage.sum(1)
+    ms = float(step_ms.mean())
+
+    # ---- end to end through the public API, host buffers (pinned), copies timed
+    x_pin = torch.from_numpy(x_h.view(np.int16)).view(torch.bfloat16).pin_memory()
+    lg_pin = torch.from_numpy(lg_h).pin_memory()
+    y_pin = torch.empty(cfg.T, cfg.H, dtype=torch.float32).pin_memory()
+    x_d = torch.empty_like(x)
+    lg_d = torch.empty_like(logits)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x_d.copy_(x_pin, non_blocking=True)
+        lg_d.copy_(lg_pin, non_blocking=True)
+        gq4.moe_expert_ffn(Wg, Wu, Wd, lg_d, x_d, cfg.K, y=y, ws=ws)
+        y_pin.copy_(y, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = float(np.mean(e2e_ms))
+
+    t = torch.tensor([ms, e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, e2e = float(t[0]), float(t[1])
+
+    hbm, bf16, peak_kind = peaks()
+    ab = alg_bytes(cfg, n_active)
+    t_gu = float(stage[:, 1].mean())
+    t_dn = float(stage[:, 2].mean())
+    dominant = ("gate_up", t_gu) if t_gu >= t_dn else ("down", t_dn)
+    achieved = ab[dominant[0]] / (dominant[1] * 1e-3) / 1e9
+    traffic = None
+    if os.path.exists(PROFILE_TRAFFIC):
+        with open(PROFILE_TRAFFIC) as f:
+            tr = json.load(f)
+        rec = tr.get(f"{cfg.name}:{dominant[0]}")
+        if rec and rec.get("source_hash") == kernel_source_hash():
+            traffic = rec["bytes_per_launch"]
+
+    if rank == 0:
+        line = {
+            "metric": "expert-FFN tokens/s (MoE layer, 1 B200)", "value": world * cfg.T / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "F": cfg.F, "K": cfg.K,
+                       "gs": 64, "distinct_experts": n_active, "parallelism": f"replicas x{world}",
+                       "l2": f"{L2_FLUSH_BYTES >> 20} MiB flush between steps; touched weights "
+                             f"{n_active * 21233664 / 1e9:.2f} GB/step > L2"},
+            "hbm_gbs_step": ab["step"] / (ms * 1e-3) / 1e9,
+            "hbm_frac_of_8tbs": ab["step"] / (ms * 1e-3) / 8e12,
+            "stage_ms": {"route_rowmap": float(stage[:, 0].mean()), "gate_up": t_gu, "down": t_dn},
+            "roofline": {"kernel": f"gq4_skinny_kernel ({dominant[0]})", "bound": "hbm",
+                         "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": traffic,
+                         "alg_bytes_per_launch": ab[dominant[0]]},
+            "e2e": {"value": world * cfg.T / (e2e * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x_h.nbytes + lg_h.nbytes, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

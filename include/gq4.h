@@ -1,0 +1,201 @@
+/*
+ * gq4.h -- C ABI of libgq4: grouped-int4 (fmt=4, gs=64) weight-only products for the
+ * routed experts of a mixture-of-experts FFN, on one NVIDIA B200 (sm_100a).
+ *
+ * Format (colibri PR #298 "cuda+engine: full fmt=4 (grouped int4 gs=64) support",
+ * sections "Changes" and "CUDA fmt=4 support ... implementation complete but blocked"):
+ *   - a matrix of `out` rows and `in` columns stores signed 4-bit weights q in -8..7,
+ *     two per byte, row-major, ceil(in/2) bytes per row; the even column sits in the low
+ *     nibble; nibbles are two's complement on the device (offset-binary host data is
+ *     converted by XOR 0x88 per byte at upload);
+ *   - one f32 scale per `gs` consecutive inputs of each row: scales[o*ng + k/gs] with
+ *     ng = ceil(in/gs), so w[o][k] = scales[o*ng + k/gs] * q[o][k].
+ *
+ * Conventions shared by every call:
+ *   - The caller owns all memory.  Device buffers are passed as raw device pointers and
+ *     host buffers as raw host pointers; nothing here allocates or frees device memory.
+ *   - Compute calls are asynchronous on the given stream (NULL = the legacy default
+ *     stream) and return after the launches are queued.
+ *   - Arguments are validated on the host before anything is launched; a call that
+ *     returns an error has launched nothing and written no output.
+ *   - Device pointers must be 16-byte aligned.  Inputs and outputs must not overlap
+ *     (pxq_llama.cpp release notes 2026-09-02, "Host-overhead cuts": the router aliasing
+ *     barrier; "Correctness fixes": a fused path that did not check 16-byte base
+ *     alignment faulted instead of declining -- here the call declines).
+ *   - The GPU kernels take gs = 64 and in % 64 == 0; other group sizes and partial last
+ *     groups return GQ4_ERR_UNSUPPORTED (the host packer accepts any shape).
+ *   - No call keeps global mutable state, reads environment variables or throws.
+ */
+#ifndef GQ4_H
+#define GQ4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GQ4_ABI_VERSION 1u
+
+typedef struct CUstream_st *gq4_stream_t; /* binary-compatible with cudaStream_t */
+typedef struct CUevent_st *gq4_event_t;   /* binary-compatible with cudaEvent_t */
+
+typedef enum {
+    GQ4_OK = 0,
+    GQ4_ERR_NULL = 1,        /* a required pointer is NULL */
+    GQ4_ERR_ALIGN = 2,       /* a device pointer or stride is not 16-byte aligned */
+    GQ4_ERR_SHAPE = 3,       /* inconsistent or out-of-range sizes */
+    GQ4_ERR_UNSUPPORTED = 4, /* valid format the GPU kernels do not take (gs != 64 ...) */
+    GQ4_ERR_ALIAS = 5,       /* an output overlaps an input */
+    GQ4_ERR_WORKSPACE = 6,   /* workspace too small */
+    GQ4_ERR_CUDA = 7,        /* a CUDA runtime call failed */
+    GQ4_ERR_TIMEOUT = 8,     /* reserved: a bounded device wait gave up */
+    GQ4_ERR_NONFINITE_LOGIT = 9 /* a router row held NaN/+inf, or no finite maximum */
+} gq4_status;
+
+typedef enum { GQ4_F32 = 0, GQ4_BF16 = 1 } gq4_dtype;
+
+/* Non-owning descriptor of one grouped-int4 matrix, or of n_experts matrices of the
+ * same shape stacked in memory (expert e at w + e*expert_stride_w bytes and
+ * s + e*expert_stride_s floats).  `w` and `s` are device pointers. */
+typedef struct {
+    int64_t out;             /* rows O */
+    int64_t in;              /* columns I (the contraction length) */
+    int32_t gs;              /* group size (64) */
+    int32_t ng;              /* ceil(in/gs) */
+    int32_t n_experts;       /* 1 for a plain matrix */
+    int32_t reserved;
+    const uint8_t *w;        /* packed nibbles [n_experts][out][ceil(in/2)] */
+    const float *s;          /* scales [n_experts][out][ng] */
+    int64_t expert_stride_w; /* bytes between experts (>= out*ceil(in/2), multiple of 16) */
+    int64_t expert_stride_s; /* floats between experts (>= out*ng, multiple of 4) */
+} gq4_tensor;
+
+/* Device views into a moe_expert_ffn workspace (see moe_expert_ffn_routing). */
+typedef struct {
+    int32_t *idx;      /* [T][K] expert of slot (t,j), logit-descending */
+    float *wts;        /* [T][K] routing weight of slot (t,j) */
+    int32_t *cnt;      /* [E] rows per expert */
+    int32_t *offs;     /* [E+1] first row of each expert; offs[E] = T*K */
+    int32_t *row_tok;  /* [T*K] token of row r */
+    int32_t *row_slot; /* [T*K] flat slot t*K+j of row r */
+    int32_t *slot_row; /* [T*K] row of flat slot f */
+    int32_t *n_active; /* [1] number of experts with cnt > 0 */
+    int32_t *active;   /* [E] those experts, ascending */
+    int32_t *status;   /* [1] device status word (gq4_status bits, see moe_expert_ffn) */
+} gq4_routing;
+
+/* ABI version of the loaded library (GQ4_ABI_VERSION at build time).  The Python
+ * binding refuses a library whose version differs (colibri PR #298, "fmt=4 CUDA
+ * attention crash": a DLL and an engine built from different branches resolved the
+ * same symbol with different signatures). */
+uint32_t gq4_abi_version(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char *gq4_status_string(int status);
+
+/* ---------------------------------------------------------------- host packing
+ * gq4_pack: q[out][in] (int8, each in -8..7 unless src_offset_binary, then 0..15
+ * offset-binary nibbles u = q+8) -> packed_host[out][ceil(in/2)], even column in the
+ * low nibble, two's complement, the pad nibble of an odd `in` written as 0.
+ * Host pointers; gs only checked (> 0).  GQ4_ERR_SHAPE on a value out of range
+ * (nothing is guaranteed written then). */
+gq4_status gq4_pack(const int8_t *q, int64_t out, int64_t in, int32_t gs,
+                    int32_t src_offset_binary, uint8_t *packed_host);
+
+/* Bytes a device copy needs: w_bytes = n_experts*out*ceil(in/2), s_bytes =
+ * n_experts*out*ceil(in/gs)*4 (colibri PR #298: qt_bytes counts O*ng*4 scale bytes). */
+gq4_status gq4_device_bytes(int64_t out, int64_t in, int32_t gs, int32_t n_experts,
+                            size_t *w_bytes, size_t *s_bytes);
+
+/* Copy packed weights and scales of n_experts matrices from host memory into
+ * caller-owned device buffers and fill *desc (expert strides = the tight sizes).  With
+ * src_offset_binary = 1 each byte is XORed with 0x88 on the device after the copy
+ * (offset_to_signed_s4).  Asynchronous on `stream`; the host buffers must stay valid
+ * until the stream reaches this point.  Device buffers must be at least the sizes from
+ * gq4_device_bytes and 16-byte aligned. */
+gq4_status gq4_upload(const uint8_t *packed_host, const float *scales_host, int64_t out,
+                      int64_t in, int32_t gs, int32_t n_experts, int32_t src_offset_binary,
+                      void *d_w, size_t d_w_bytes, float *d_s, size_t d_s_bytes,
+                      gq4_stream_t stream, gq4_tensor *desc);
+
+/* Fill *desc for device data already laid out as above (no copy). */
+gq4_status gq4_tensor_init(const void *d_w, const float *d_s, int64_t out, int64_t in,
+                           int32_t gs, int32_t n_experts, gq4_tensor *desc);
+
+/* ---------------------------------------------------------------- compute
+ * gq4_matvec: y[t][o] = sum_k w[o][k] * x[t][k] for t < n_tok, fp32 accumulation
+ * (colibri PR #298, "Changes": quant_matmul with per-group scales; the maintainer's
+ * reply: matmul_i4_grouped against a double reference).
+ *   W: one matrix (n_experts == 1); x: device [n_tok][W->in] of xdt; y: device f32
+ *   [n_tok][W->out].  f32 x is taken exactly (split into three bf16 terms).
+ *   Any n_tok >= 1; the kernel is built for few tokens (decode). */
+gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t n_tok,
+                      float *y, gq4_stream_t stream);
+
+/* gq4_gate_up_silu: g = Wg x, u = Wu x in one pass over x (x read once), then
+ * h = silu(g) * u = g * sigmoid(g) * u, rounded to xdt (bf16 round-to-nearest-even, or
+ * f32).  colibri PR #298, "Changes": matmul_i4_grouped_pair, "fused gate+up for fmt=4
+ * -- reads x once instead of twice".
+ *   Wg, Wu: one matrix each, same shape [F][H]; x device [n_tok][H] xdt; h device
+ *   [n_tok][F] xdt. */
+gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const void *x,
+                            gq4_dtype xdt, int64_t n_tok, void *h, gq4_stream_t stream);
+
+/* gq4_route: router top-K and weights, per token (colibri PR #298, "implementation
+ * complete but blocked": K passes over a taken-flag array; ties go to the lower expert
+ * index).  wts = softmax over all E renormalised over the K chosen.
+ *   logits device f32 [T][E]; idx device int32 [T][K]; wts device f32 [T][K];
+ *   status device int32 [1]: GQ4_ERR_NONFINITE_LOGIT is OR-ed in when a row holds NaN or
+ *   +inf or has no finite maximum (that row gets experts 0..K-1 and NaN weights).
+ *   1 <= K <= E <= 1024. */
+gq4_status gq4_route(const float *logits, int64_t T, int32_t E, int32_t K, int32_t *idx,
+                     float *wts, int32_t *status, gq4_stream_t stream);
+
+/* gq4_rowmap: on-device token -> expert table (pxq_llama.cpp release notes 2026-09-02,
+ * "Device-side MoE row map": histogram, scan and fill with no host round trip).
+ * Rows of an expert are ordered by ascending flat slot f = t*K + j.  Writes cnt [E],
+ * offs [E+1], row_tok / row_slot / slot_row [T*K], n_active [1], active [E] (device).
+ * `scratch` is device memory of gq4_rowmap_scratch_bytes(T, K, E) bytes. */
+size_t gq4_rowmap_scratch_bytes(int64_t T, int32_t K, int32_t E);
+gq4_status gq4_rowmap(const int32_t *idx, int64_t T, int32_t K, int32_t E, int32_t *cnt,
+                      int32_t *offs, int32_t *row_tok, int32_t *row_slot, int32_t *slot_row,
+                      int32_t *n_active, int32_t *active, void *scratch, size_t scratch_bytes,
+                      gq4_stream_t stream);
+
+/* moe_expert_ffn: one routed-expert FFN layer.
+ *   y[t] = sum_j wts[t][j] * Wd_e (silu(Wg_e x_t) * (Wu_e x_t)),  e = idx[t][j]
+ * with the router, the on-device row map, the fused gate+up (h rounded to bf16), the
+ * down projection and the weighted scatter-add all on the GPU, no host round trip.
+ *   Wg, Wu: E stacked [F][H]; Wd: E stacked [H][F]; logits device f32 [T][E];
+ *   x device bf16 [T][H]; y device f32 [T][H] (overwritten); ws device workspace of
+ *   moe_expert_ffn_workspace_bytes(T, E, K, H, F) bytes; 1 <= K <= E <= 1024.
+ * Data-dependent errors (non-finite logits) are reported through the workspace status
+ * word: read it with moe_expert_ffn_status.  The order in which the K slot
+ * contributions are added into y is not fixed (float atomics); results agree within
+ * rounding.
+ *   stage_events: NULL, or 4 CUDA events (created by the caller) recorded on `stream`
+ *   at the start, after the router and row map, after gate+up and after down, so a
+ *   caller can time the stages with cudaEventElapsedTime. */
+size_t moe_expert_ffn_workspace_bytes(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F);
+gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_tensor *Wd,
+                          const float *logits, const void *x, gq4_dtype xdt, int64_t T,
+                          int32_t E, int32_t K, float *y, void *ws, size_t ws_bytes,
+                          gq4_event_t const *stage_events, gq4_stream_t stream);
+
+/* Device pointers of the routing tables inside a workspace used by moe_expert_ffn with
+ * the same (T, E, K, H, F). */
+gq4_status moe_expert_ffn_routing(void *ws, size_t ws_bytes, int64_t T, int32_t E, int32_t K,
+                                  int64_t H, int64_t F, gq4_routing *out);
+
+/* Synchronise `stream` and read the workspace status word into *status (GQ4_OK when no
+ * data error was seen).  Returns GQ4_ERR_CUDA when the synchronisation fails. */
+gq4_status moe_expert_ffn_status(const void *ws, size_t ws_bytes, int64_t T, int32_t E,
+                                 int32_t K, int64_t H, int64_t F, gq4_stream_t stream,
+                                 int32_t *status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GQ4_H */

@@ -1,0 +1,280 @@
+"""GPU parity: every call of the C ABI against the CPU oracle on the same seeded inputs.
+
+Routing and the row map are compared bit for bit; floating-point outputs within
+|err| <= 2e-3 * (sum of |terms|) per element and relative L2 <= 1e-4."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.helpers import (bf16_to_torch, check_bf16_close, check_close, h_bound,
+                           torch_bf16_to_bits)
+from weight_only_int4_gq4_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from weight_only_int4_gq4_b200 import gq4
+
+
+def _x_torch(x):
+    return bf16_to_torch(x) if x.dtype == np.uint16 else torch.from_numpy(x).cuda()
+
+
+# ---------------------------------------------------------------- a1-a2 matvec
+MV_CASES = [
+    # O, I, T, dtype  -- several tiles, ragged row tails, 1..40 tokens, f32 and bf16 x
+    (16, 64, 1, "bf16"), (50, 256, 1, "bf16"), (200, 640, 3, "f32"), (33, 1024, 9, "bf16"),
+    (64, 512, 20, "bf16"), (16, 128, 40, "bf16"), (100, 4096, 1, "f32"), (7, 192, 2, "f32"),
+    (1000, 1536, 5, "bf16"), (24, 64, 11, "f32"),
+]
+
+
+@pytest.mark.parametrize("O,I,T,dt", MV_CASES)
+def test_matvec_small(O, I, T, dt):
+    q = synth.q_uniform(31, O, I, O, I, T)
+    s = synth.scales_uniform(31, O, I // 64, -0.02, 0.02, O, I, T)
+    x = synth.x_normal(31, T, I, dt, O, I, T)
+    W = gq4.upload(gq4.pack(q), s)
+    y = gq4.matvec(W, _x_torch(x)).cpu().numpy()
+    y_orc, bound = oracle.matvec(oracle.pack(q), s, x)
+    check_close(y, y_orc, bound, f"matvec {O}x{I} T={T} {dt}")
+
+
+def test_matvec_scale_extremes_and_nibble_extremes():
+    O, I = 48, 256
+    for byte in (0x77, 0x88, 0x00, 0xF8):
+        p = np.full((O, I // 2), byte, np.uint8)
+        s = np.tile(np.array([0.0, -1.5, 1e-3, 3e4], np.float32), (O, 1))
+        x = synth.x_normal(2, 2, I, "bf16")
+        y = gq4.matvec(gq4.upload(p, s), bf16_to_torch(x)).cpu().numpy()
+        y_orc, bound = oracle.matvec(p, s, x)
+        check_close(y, y_orc, bound, f"byte {byte:#x}")
+
+
+def test_matvec_offset_binary_upload():
+    O, I = 32, 128
+    q = synth.q_uniform(5, O, I)
+    s = synth.scales_uniform(5, O, 2, 0.002, 0.02)
+    u = (q.astype(np.int16) + 8).astype(np.int8)
+    pob = oracle.pack(q, offset_binary=True)           # host file in offset binary
+    assert np.array_equal(gq4.pack(u, offset_binary=True), oracle.pack(q))
+    W = gq4.upload(pob, s, offset_binary=True)         # XOR 0x88 on the device
+    assert np.array_equal(W.w.cpu().numpy().reshape(O, I // 2), oracle.pack(q))
+    x = synth.x_normal(5, 1, I, "bf16")
+    check_close(gq4.matvec(W, bf16_to_torch(x)).cpu().numpy(), *oracle.matvec(oracle.pack(q), s, x))
+
+
+@pytest.mark.parametrize("O,I", synth.DENSE_SHAPES)
+def test_matvec_dense_sweep_full_size(O, I):
+    """The dense sweep at full size, in the launch configuration the benchmark uses;
+    the oracle checks every row (largest shape: a seeded sample of 4096 rows)."""
+    p, s, x = synth.dense_matvec(O, I)
+    W = gq4.upload(p, s)
+    y = gq4.matvec(W, bf16_to_torch(x)).cpu().numpy()
+    rows = np.arange(O) if O * I <= 14336 * 4096 else np.sort(
+        np.random.default_rng(O).choice(O, 4096, replace=False))
+    y_orc, bound = oracle.matvec(p[rows], s[rows], x)
+    check_close(y[:, rows], y_orc, bound, f"dense {O}x{I}")
+
+
+# ---------------------------------------------------------------- a3 gate+up+SiLU
+def test_single_expert_f32():
+    """1024 -> 2048 -> 1024, x f32: fused gate+up+SiLU then down."""
+    c = synth.SingleExpert()
+    Wg = gq4.upload(gq4.pack(c.qg), c.sg)
+    Wu = gq4.upload(gq4.pack(c.qu), c.su)
+    Wd = gq4.upload(gq4.pack(c.qd), c.sd)
+    x = torch.from_numpy(c.x).cuda()
+    h = gq4.gate_up_silu(Wg, Wu, x)
+    y = gq4.matvec(Wd, h).cpu().numpy()
+    pg, pu, pd = oracle.pack(c.qg), oracle.pack(c.qu), oracle.pack(c.qd)
+    h_orc, g, u = oracle.gate_up_silu(pg, c.sg, pu, c.su, c.x)
+    hb = h_bound(oracle.row_l1(pg, c.sg, c.H), oracle.row_l1(pu, c.su, c.H), np.abs(c.x).max(1), g, u)
+    check_close(h.cpu().numpy(), h_orc, hb, "h (f32)")
+    y_orc, bound = oracle.matvec(pd, c.sd, h_orc.astype(np.float32))
+    check_close(y, y_orc, bound, "y")
+    # pair invariant on the GPU: fused gate+up == two separate matvecs
+    g_gpu = gq4.matvec(Wg, x).cpu().numpy()
+    u_gpu = gq4.matvec(Wu, x).cpu().numpy()
+    check_close(g_gpu, g, oracle.matvec(pg, c.sg, c.x)[1], "g")
+    check_close(u_gpu, u, oracle.matvec(pu, c.su, c.x)[1], "u")
+
+
+@pytest.mark.parametrize("F,H,T", [(48, 256, 1), (2048, 1024, 3), (160, 4096, 12), (64, 512, 33)])
+def test_gate_up_silu_bf16(F, H, T):
+    qg, qu = synth.q_uniform(8, F, H, 0), synth.q_uniform(8, F, H, 1)
+    sg = synth.scales_uniform(8, F, H // 64, 0.002, 0.02, 0)
+    su = synth.scales_uniform(8, F, H // 64, 0.002, 0.02, 1)
+    x = synth.x_normal(8, T, H, "bf16")
+    h = gq4.gate_up_silu(gq4.upload(gq4.pack(qg), sg), gq4.upload(gq4.pack(qu), su), bf16_to_torch(x))
+    pg, pu = oracle.pack(qg), oracle.pack(qu)
+    h_orc, g, u = oracle.gate_up_silu(pg, sg, pu, su, x)
+    xm = np.abs(synth.bf16_bits_to_f32(x)).max(1)
+    hb = h_bound(oracle.row_l1(pg, sg, H), oracle.row_l1(pu, su, H), xm, g, u)
+    check_bf16_close(torch_bf16_to_bits(h), h_orc, hb, f"h {F}x{H} T={T}")
+
+
+# ---------------------------------------------------------------- a4 router, a5 row map
+def _route_both(lg, K):
+    st, idx_o, wts_o, bad = oracle.route(lg, K)
+    idx, wts, status = gq4.route(torch.from_numpy(lg).cuda(), K)
+    return (st, idx_o, wts_o, bad), (idx.cpu().numpy(), wts.cpu().numpy(), int(status.cpu()[0]))
+
+
+@pytest.mark.parametrize("T,E,K", [(1, 128, 8), (32, 256, 8), (7, 4, 4), (100, 16, 2), (5, 1000, 8),
+                                   (3, 33, 1), (64, 64, 64)])
+def test_route_bitexact(T, E, K):
+    lg, _ = synth.logits_normal(T * E + K, T, E)
+    lg[:, ::7] = np.round(lg[:, ::7])  # plenty of exact ties
+    (st, idx_o, wts_o, bad), (idx, wts, status) = _route_both(lg, K)
+    assert st == oracle.OK and status == 0
+    assert np.array_equal(idx, idx_o)
+    assert np.allclose(wts, wts_o, rtol=1e-6, atol=0)
+
+
+def test_route_nonfinite_rows():
+    lg, _ = synth.logits_normal(9, 6, 40)
+    lg[1, 3] = np.nan
+    lg[2, :] = -np.inf
+    lg[4, 7] = np.inf
+    lg[5, :20] = -np.inf
+    (st, idx_o, wts_o, bad), (idx, wts, status) = _route_both(lg, 4)
+    assert st == oracle.ERR_NONFINITE_LOGIT and status == oracle.ERR_NONFINITE_LOGIT
+    assert np.array_equal(idx, idx_o)
+    ok = bad == 0
+    assert np.allclose(wts[ok], wts_o[ok], rtol=1e-6, atol=0)
+    assert np.all(np.isnan(wts[~ok]))
+
+
+ROWMAP_CASES = [(T, E, K) for T, E, K in
+                [(1, 128, 8), (32, 256, 8), (4096, 256, 8), (7, 4, 4), (129, 16, 8), (1000, 1024, 3),
+                 (300, 64, 2), (513, 8, 2), (64, 64, 64), (2, 5, 1)]] + \
+               [(int(t), int(e), int(k)) for t, e, k in
+                np.random.default_rng(64).integers([1, 2, 1], [2000, 300, 9], size=(54, 3))]
+
+
+@pytest.mark.parametrize("T,E,K", ROWMAP_CASES)
+def test_rowmap_bitexact(T, E, K):
+    K = min(K, E)
+    lg, _ = synth.logits_normal(T + 7 * E + K, T, E, sigma=1.0, n_hot=min(4, E), hot_bias=2.0)
+    st, idx_o, _, _ = oracle.route(lg, K)
+    m_o = oracle.rowmap(idx_o, E)
+    m = gq4.rowmap(torch.from_numpy(idx_o).cuda(), E)
+    for k in ("cnt", "offs", "row_tok", "row_slot", "slot_row"):
+        assert np.array_equal(m[k].cpu().numpy(), m_o[k]), k
+    act = np.nonzero(m_o["cnt"])[0]
+    assert int(m["n_active"].cpu()[0]) == len(act)
+    assert np.array_equal(m["active"].cpu().numpy()[:len(act)], act)
+    assert int(m["status"].cpu()[0]) == 0
+
+
+def test_rowmap_rejects_bad_index():
+    idx = torch.tensor([[0, 1], [2, 9]], dtype=torch.int32, device="cuda")
+    m = gq4.rowmap(idx, 4)
+    assert int(m["status"].cpu()[0]) == oracle.ERR_SHAPE
+
+
+# ---------------------------------------------------------------- a6-a8 MoE layer
+class MoESet:
+    """Stacked experts of one workload on the host (packed bytes, scales) and the GPU."""
+
+    def __init__(self, cfg: synth.MoEConfig):
+        self.cfg = cfg
+        E = cfg.E
+        gate = [cfg.gate(e) for e in range(E)]
+        up = [cfg.up(e) for e in range(E)]
+        down = [cfg.down(e) for e in range(E)]
+        self.pg = np.stack([a for a, _ in gate]); self.sg = np.stack([b for _, b in gate])
+        self.pu = np.stack([a for a, _ in up]); self.su = np.stack([b for _, b in up])
+        self.pd = np.stack([a for a, _ in down]); self.sd = np.stack([b for _, b in down])
+        del gate, up, down
+        self.Wg = gq4.upload(self.pg, self.sg)
+        self.Wu = gq4.upload(self.pu, self.su)
+        self.Wd = gq4.upload(self.pd, self.sd)
+        self.lg, self.hot = cfg.logits()
+        self.x = cfg.x()
+
+    def run(self, lg=None):
+        lg = self.lg if lg is None else lg
+        y, ws = gq4.moe_expert_ffn(self.Wg, self.Wu, self.Wd, torch.from_numpy(lg).cuda(),
+                                   bf16_to_torch(self.x), self.cfg.K)
+        return y.cpu().numpy(), ws
+
+    def check(self, y, ws, tokens, lg=None):
+        cfg = self.cfg
+        lg = self.lg if lg is None else lg
+        st, idx_o, wts_o, bad = oracle.route(lg, cfg.K)
+        r = ws.routing()
+        assert np.array_equal(r["idx"].cpu().numpy(), idx_o)
+        ok = bad == 0
+        assert np.allclose(r["wts"].cpu().numpy()[ok], wts_o[ok], rtol=1e-6, atol=0)
+        m_o = oracle.rowmap(idx_o, cfg.E)
+        for k in ("cnt", "offs", "row_tok", "row_slot", "slot_row"):
+            assert np.array_equal(r[k].cpu().numpy(), m_o[k]), k
+        tokens = np.asarray([t for t in tokens if ok[t]], np.int64)
+        y_orc, bound = oracle.moe_tokens(self.pg, self.sg, self.pu, self.su, self.pd, self.sd, cfg.H,
+                                         cfg.F, self.x, idx_o, wts_o, tokens)
+        return check_close(y[tokens], y_orc, bound, cfg.name)
+
+
+def _toy(T, E, K, H=128, F=128, seed=3, **kw):
+    return synth.MoEConfig(f"toy_t{T}_e{E}_k{K}", T=T, H=H, E=E, F=F, K=K, seed=seed, **kw)
+
+
+@pytest.mark.parametrize("T,E,K,H,F", [(5, 4, 2, 128, 128), (1, 1, 1, 64, 64), (3, 8, 8, 192, 256),
+                                       (17, 16, 4, 256, 128), (40, 32, 8, 128, 192),
+                                       (300, 16, 4, 128, 64)])
+def test_moe_small_full_oracle(T, E, K, H, F):
+    s = MoESet(_toy(T, E, K, H, F))
+    y, ws = s.run()
+    assert ws.status() == 0
+    s.check(y, ws, np.arange(T))
+
+
+def test_moe_nonfinite_logits_flagged():
+    s = MoESet(_toy(6, 8, 2))
+    lg = s.lg.copy()
+    lg[2, 5] = np.nan
+    y, ws = s.run(lg)
+    assert ws.status() == oracle.ERR_NONFINITE_LOGIT
+    assert np.all(np.isnan(y[2]))
+    s.check(y, ws, [0, 1, 3, 4, 5], lg)
+
+
+@pytest.fixture(scope="module")
+def moe_decode():
+    return MoESet(synth.MOE_DECODE)
+
+
+def test_moe_decode_full_size(moe_decode):
+    y, ws = moe_decode.run()
+    assert ws.status() == 0
+    moe_decode.check(y, ws, np.arange(1))
+
+
+def test_moe_batched_decode_full_size():
+    """The benchmark's workload (32 tokens, 256 experts of 6144 x 2048, top-8, skewed
+    routing), in the benchmark's launch configuration; routing and the row map in
+    full, the output on a seeded sample of 8 tokens."""
+    s = MoESet(synth.MOE_BATCHED)
+    y, ws = s.run()
+    assert ws.status() == 0
+    y2, _ = s.run()  # a second call reuses nothing stale
+    assert np.allclose(y, y2, rtol=1e-5, atol=1e-3)
+    tokens = np.sort(np.random.default_rng(1003).choice(32, 8, replace=False))
+    s.check(y, ws, tokens)
+    del s
+    torch.cuda.empty_cache()
+
+
+def test_moe_prefill_full_size():
+    """4096 tokens over all 256 experts; routing and the row map in full, the output
+    on 4 tokens of the seeded 256-token sample."""
+    s = MoESet(synth.MOE_PREFILL)
+    y, ws = s.run()
+    assert ws.status() == 0
+    tokens = synth.MOE_PREFILL.sample_tokens()[::64]
+    s.check(y, ws, tokens)
+    del s
+    torch.cuda.empty_cache()

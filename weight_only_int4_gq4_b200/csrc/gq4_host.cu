@@ -1,0 +1,531 @@
+// gq4_host.cu -- the C ABI of libgq4 (declared in include/gq4.h): argument checks,
+// workspace layout and kernel launches.  Every compute step runs in the kernels of
+// gq4_skinny.cuh / gq4_route.cuh / gq4_prefill.cuh; this file only validates and
+// launches.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "gq4.h"
+#include "gq4_common.cuh"
+#include "gq4_route.cuh"
+#include "gq4_skinny.cuh"
+
+using namespace gq4;
+
+namespace {
+
+inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;
+};
+inline Range rng(const void *p, size_t bytes) { return {(uintptr_t)p, (uintptr_t)p + bytes}; }
+inline bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+inline cudaStream_t S(gq4_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Checks of one tensor descriptor for the GPU kernels.
+gq4_status check_tensor(const gq4_tensor *t, int n_experts_min) {
+    if (!t || !t->w || !t->s) return GQ4_ERR_NULL;
+    if (t->out < 1 || t->in < 1 || t->n_experts < n_experts_min) return GQ4_ERR_SHAPE;
+    if (t->gs <= 0 || t->ng != (t->in + t->gs - 1) / t->gs) return GQ4_ERR_SHAPE;
+    if (t->gs != kGroup || t->in % kGroup != 0) return GQ4_ERR_UNSUPPORTED;
+    if (t->out > (int64_t)1 << 30 || t->in > (int64_t)1 << 20) return GQ4_ERR_SHAPE;
+    if (!aligned16(t->w) || !aligned16(t->s)) return GQ4_ERR_ALIGN;
+    if (t->n_experts > 1) {
+        if (t->expert_stride_w < t->out * (t->in / 2) || t->expert_stride_s < t->out * t->ng)
+            return GQ4_ERR_SHAPE;
+        if (t->expert_stride_w % 16 || t->expert_stride_s % 4) return GQ4_ERR_ALIGN;
+    }
+    return GQ4_OK;
+}
+
+inline size_t tensor_w_bytes(const gq4_tensor *t) {
+    return (size_t)(t->n_experts - 1) * t->expert_stride_w + (size_t)t->out * (t->in / 2);
+}
+inline size_t tensor_s_bytes(const gq4_tensor *t) {
+    return ((size_t)(t->n_experts - 1) * t->expert_stride_s + (size_t)t->out * t->ng) * 4;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory (once per process; the
+// attribute applies to the function in every context of the process).
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)std::min<size_t>(bytes, 227 * 1024));
+}
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+// ---- skinny launches -----------------------------------------------------------------
+size_t skinny_smem(int mode_pair, int NT, int xcols, int I) {
+    return (size_t)xcols * skinny_xstride(I) + (size_t)8 * mode_pair * 16 * NT * 8 * 4;
+}
+
+template <int MODE, int NT>
+gq4_status launch_skinny_nt(const SkinnyParams &p, int units_upper, cudaStream_t st) {
+    constexpr int PAIR = ModeTraits<MODE>::kPair;
+    constexpr int UG = PAIR == 2 ? 2 : 4;
+    auto kern = gq4_skinny_kernel<MODE, NT, UG>;
+    const size_t smem = skinny_smem(PAIR, NT, p.xcols, p.I);
+    if (smem > kMaxSmem) return GQ4_ERR_UNSUPPORTED;
+    if (allow_smem(kern, smem) != cudaSuccess) return GQ4_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess)
+        return GQ4_ERR_CUDA;
+    per_sm = std::max(per_sm, 1);
+    const int grid = std::max(1, std::min(units_upper, per_sm * sm_count()));
+    kern<<<grid, 256, smem, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
+// Choose the n-tile count and the staged-column budget for `cols` columns per unit.
+template <int MODE>
+gq4_status launch_skinny(SkinnyParams p, int max_cols, bool f32x, int units_upper, cudaStream_t st) {
+    constexpr int PAIR = ModeTraits<MODE>::kPair;
+    int NT = max_cols <= 8 ? 1 : (max_cols <= 16 ? 2 : 4);
+    // staged columns: as many as fit next to the reduction buffer (at most ~96 KB so two
+    // CTAs share an SM), a multiple of 3 for f32 activations, at least one pass
+    const size_t red = (size_t)8 * PAIR * 16 * NT * 8 * 4;
+    const size_t xs = skinny_xstride(p.I);
+    size_t budget = 96 * 1024 > red ? 96 * 1024 - red : 0;
+    int fit = (int)std::min<size_t>(budget / xs, 1 << 20);
+    int xcols = std::min(max_cols, std::max(fit, f32x ? 3 : 1));
+    if (f32x) xcols = std::max(3, xcols / 3 * 3);
+    if ((size_t)xcols * xs + red > kMaxSmem) return GQ4_ERR_UNSUPPORTED;
+    p.xcols = xcols;
+    switch (NT) {
+        case 1: return launch_skinny_nt<MODE, 1>(p, units_upper, st);
+        case 2: return launch_skinny_nt<MODE, 2>(p, units_upper, st);
+        default: return launch_skinny_nt<MODE, 4>(p, units_upper, st);
+    }
+}
+
+// ---- MoE workspace layout --------------------------------------------------------------
+struct MoeLayout {
+    size_t status, idx, wts, cnt, offs, row_tok, row_slot, slot_row, n_active, active, chunk,
+        h, total;
+};
+
+inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+MoeLayout moe_layout(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F) {
+    (void)H;
+    MoeLayout L{};
+    const size_t n = (size_t)T * K;
+    const size_t nchunks = (n + kChunk - 1) / kChunk;
+    size_t o = 0;
+    L.status = o; o = al256(o + 16);
+    L.idx = o; o = al256(o + n * 4);
+    L.wts = o; o = al256(o + n * 4);
+    L.cnt = o; o = al256(o + (size_t)E * 4);
+    L.offs = o; o = al256(o + (size_t)(E + 1) * 4);
+    L.row_tok = o; o = al256(o + n * 4);
+    L.row_slot = o; o = al256(o + n * 4);
+    L.slot_row = o; o = al256(o + n * 4);
+    L.n_active = o; o = al256(o + 16);
+    L.active = o; o = al256(o + (size_t)E * 4);
+    L.chunk = o; o = al256(o + nchunks * (size_t)E * 4);
+    L.h = o; o = al256(o + n * (size_t)F * 2);
+    L.total = o;
+    return L;
+}
+
+template <typename T>
+inline T *at(void *ws, size_t off) { return reinterpret_cast<T *>((char *)ws + off); }
+
+int epl_for(int E) {
+    int epl = 1;
+    while (epl * 32 < E) epl *= 2;
+    return epl;
+}
+
+gq4_status launch_route(const float *logits, int T, int E, int K, int32_t *idx, float *wts,
+                        int32_t *status, cudaStream_t st) {
+    const int grid = (T + 7) / 8;
+    switch (epl_for(E)) {
+#define ROUTE_CASE(N) case N: gq4_route_kernel<N><<<grid, 256, 0, st>>>(logits, T, E, K, idx, wts, status); break;
+        ROUTE_CASE(1) ROUTE_CASE(2) ROUTE_CASE(4) ROUTE_CASE(8) ROUTE_CASE(16) ROUTE_CASE(32)
+#undef ROUTE_CASE
+        default: return GQ4_ERR_SHAPE;
+    }
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
+gq4_status launch_rowmap(const int32_t *idx, int n, int K, int E, int32_t *cnt, int32_t *offs,
+                         int32_t *row_tok, int32_t *row_slot, int32_t *slot_row, int32_t *n_active,
+                         int32_t *active, int32_t *chunk, int32_t *status, cudaStream_t st) {
+    const int nchunks = (n + kChunk - 1) / kChunk;
+    gq4_rowmap_count_kernel<<<nchunks, kChunk, 0, st>>>(idx, n, E, chunk, status);
+    gq4_rowmap_scan_kernel<<<1, 1024, 0, st>>>(chunk, nchunks, E, cnt, offs, n_active, active);
+    const size_t smem = (size_t)32 * E * 4;
+    if (allow_smem(gq4_rowmap_fill_kernel, smem) != cudaSuccess) return GQ4_ERR_CUDA;
+    gq4_rowmap_fill_kernel<<<nchunks, kChunk, smem, st>>>(idx, n, K, E, chunk, row_tok, row_slot,
+                                                          slot_row);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
+gq4_status launch_route_rowmap_small(const float *logits, int T, int E, int K, void *ws,
+                                     const MoeLayout &L, cudaStream_t st) {
+    const size_t smem = (size_t)33 * E * 4;
+    int32_t *status = at<int32_t>(ws, L.status);
+#define SMALL_ARGS logits, T, E, K, at<int32_t>(ws, L.idx), at<float>(ws, L.wts), status,      \
+                   at<int32_t>(ws, L.cnt), at<int32_t>(ws, L.offs), at<int32_t>(ws, L.n_active), \
+                   at<int32_t>(ws, L.active), at<int32_t>(ws, L.row_tok),                        \
+                   at<int32_t>(ws, L.row_slot), at<int32_t>(ws, L.slot_row)
+    switch (epl_for(E)) {
+#define SMALL_CASE(N)                                                                    \
+    case N:                                                                              \
+        if (allow_smem(gq4_route_rowmap_small_kernel<N>, smem) != cudaSuccess) return GQ4_ERR_CUDA; \
+        gq4_route_rowmap_small_kernel<N><<<1, 1024, smem, st>>>(SMALL_ARGS);             \
+        break;
+        SMALL_CASE(1) SMALL_CASE(2) SMALL_CASE(4) SMALL_CASE(8) SMALL_CASE(16) SMALL_CASE(32)
+#undef SMALL_CASE
+#undef SMALL_ARGS
+        default: return GQ4_ERR_SHAPE;
+    }
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
+__global__ void gq4_xor88_kernel(uint4 *p, size_t n16, uint8_t *tail, size_t ntail) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n16) {
+        uint4 v = p[i];
+        v.x ^= 0x88888888u; v.y ^= 0x88888888u; v.z ^= 0x88888888u; v.w ^= 0x88888888u;
+        p[i] = v;
+    }
+    if (i < ntail) tail[i] ^= 0x88u;
+}
+
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+uint32_t gq4_abi_version(void) { return GQ4_ABI_VERSION; }
+
+const char *gq4_status_string(int status) {
+    switch (status) {
+        case GQ4_OK: return "ok";
+        case GQ4_ERR_NULL: return "a required pointer is NULL";
+        case GQ4_ERR_ALIGN: return "a device pointer or stride is not 16-byte aligned";
+        case GQ4_ERR_SHAPE: return "inconsistent or out-of-range sizes";
+        case GQ4_ERR_UNSUPPORTED: return "format or size not supported by the GPU kernels";
+        case GQ4_ERR_ALIAS: return "an output overlaps an input";
+        case GQ4_ERR_WORKSPACE: return "workspace too small";
+        case GQ4_ERR_CUDA: return "CUDA runtime error";
+        case GQ4_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case GQ4_ERR_NONFINITE_LOGIT: return "router logits hold NaN/+inf or no finite maximum";
+        default: return "unknown status";
+    }
+}
+
+gq4_status gq4_pack(const int8_t *q, int64_t out, int64_t in, int32_t gs,
+                    int32_t src_offset_binary, uint8_t *packed_host) {
+    if (!q || !packed_host) return GQ4_ERR_NULL;
+    if (out < 0 || in < 0 || gs <= 0) return GQ4_ERR_SHAPE;
+    const int64_t rb = (in + 1) / 2;
+    for (int64_t o = 0; o < out; ++o) {
+        const int8_t *qr = q + o * in;
+        uint8_t *dst = packed_host + o * rb;
+        for (int64_t b = 0; b < rb; ++b) {
+            int lo = qr[2 * b], hi = (2 * b + 1 < in) ? qr[2 * b + 1] : 0;
+            if (src_offset_binary) {
+                if (lo < 0 || lo > 15 || hi < 0 || hi > 15) return GQ4_ERR_SHAPE;
+                lo -= 8;
+                hi = (2 * b + 1 < in) ? hi - 8 : 0;
+            } else if (lo < -8 || lo > 7 || hi < -8 || hi > 7) {
+                return GQ4_ERR_SHAPE;
+            }
+            dst[b] = (uint8_t)((lo & 15) | ((hi & 15) << 4));
+        }
+    }
+    return GQ4_OK;
+}
+
+gq4_status gq4_device_bytes(int64_t out, int64_t in, int32_t gs, int32_t n_experts,
+                            size_t *w_bytes, size_t *s_bytes) {
+    if (!w_bytes || !s_bytes) return GQ4_ERR_NULL;
+    if (out < 1 || in < 1 || gs <= 0 || n_experts < 1) return GQ4_ERR_SHAPE;
+    *w_bytes = (size_t)n_experts * out * ((in + 1) / 2);
+    *s_bytes = (size_t)n_experts * out * ((in + gs - 1) / gs) * 4;
+    return GQ4_OK;
+}
+
+gq4_status gq4_tensor_init(const void *d_w, const float *d_s, int64_t out, int64_t in,
+                           int32_t gs, int32_t n_experts, gq4_tensor *desc) {
+    if (!d_w || !d_s || !desc) return GQ4_ERR_NULL;
+    if (out < 1 || in < 1 || gs <= 0 || n_experts < 1) return GQ4_ERR_SHAPE;
+    gq4_tensor t{};
+    t.out = out;
+    t.in = in;
+    t.gs = gs;
+    t.ng = (int32_t)((in + gs - 1) / gs);
+    t.n_experts = n_experts;
+    t.w = (const uint8_t *)d_w;
+    t.s = d_s;
+    t.expert_stride_w = out * ((in + 1) / 2);
+    t.expert_stride_s = out * t.ng;
+    *desc = t;
+    return GQ4_OK;
+}
+
+gq4_status gq4_upload(const uint8_t *packed_host, const float *scales_host, int64_t out,
+                      int64_t in, int32_t gs, int32_t n_experts, int32_t src_offset_binary,
+                      void *d_w, size_t d_w_bytes, float *d_s, size_t d_s_bytes,
+                      gq4_stream_t stream, gq4_tensor *desc) {
+    if (!packed_host || !scales_host || !d_w || !d_s || !desc) return GQ4_ERR_NULL;
+    size_t wb = 0, sb = 0;
+    gq4_status st = gq4_device_bytes(out, in, gs, n_experts, &wb, &sb);
+    if (st != GQ4_OK) return st;
+    if (d_w_bytes < wb || d_s_bytes < sb) return GQ4_ERR_SHAPE;
+    if (!aligned16(d_w) || !aligned16(d_s)) return GQ4_ERR_ALIGN;
+    if (overlap(rng(d_w, wb), rng(d_s, sb))) return GQ4_ERR_ALIAS;
+    cudaStream_t s = S(stream);
+    if (cudaMemcpyAsync(d_w, packed_host, wb, cudaMemcpyHostToDevice, s) != cudaSuccess) return GQ4_ERR_CUDA;
+    if (cudaMemcpyAsync(d_s, scales_host, sb, cudaMemcpyHostToDevice, s) != cudaSuccess) return GQ4_ERR_CUDA;
+    if (src_offset_binary) {
+        const size_t n16 = wb / 16, ntail = wb % 16;
+        const size_t nthreads = std::max(n16, ntail);
+        const unsigned grid = (unsigned)((nthreads + 255) / 256);
+        if (grid) gq4_xor88_kernel<<<grid, 256, 0, s>>>((uint4 *)d_w, n16, (uint8_t *)d_w + n16 * 16, ntail);
+        if (cudaGetLastError() != cudaSuccess) return GQ4_ERR_CUDA;
+    }
+    return gq4_tensor_init(d_w, d_s, out, in, gs, n_experts, desc);
+}
+
+gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t n_tok,
+                      float *y, gq4_stream_t stream) {
+    gq4_status st = check_tensor(W, 1);
+    if (st != GQ4_OK) return st;
+    if (!x || !y) return GQ4_ERR_NULL;
+    if (xdt != GQ4_F32 && xdt != GQ4_BF16) return GQ4_ERR_UNSUPPORTED;
+    if (n_tok < 1 || n_tok > (1 << 20)) return GQ4_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(y)) return GQ4_ERR_ALIGN;
+    const size_t xb = (size_t)n_tok * W->in * (xdt == GQ4_F32 ? 4 : 2);
+    const Range yr = rng(y, (size_t)n_tok * W->out * 4);
+    if (overlap(yr, rng(x, xb)) || overlap(yr, rng(W->w, tensor_w_bytes(W))) ||
+        overlap(yr, rng(W->s, tensor_s_bytes(W))))
+        return GQ4_ERR_ALIAS;
+    SkinnyParams p{};
+    p.w0 = W->w; p.s0 = W->s;
+    p.O = (int)W->out; p.I = (int)W->in; p.ng = W->ng;
+    p.row_tiles = (int)((W->out + 15) / 16);
+    p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
+    p.y = y;
+    const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    return launch_skinny<kMatvec>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
+}
+
+gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const void *x,
+                            gq4_dtype xdt, int64_t n_tok, void *h, gq4_stream_t stream) {
+    gq4_status st = check_tensor(Wg, 1);
+    if (st != GQ4_OK) return st;
+    st = check_tensor(Wu, 1);
+    if (st != GQ4_OK) return st;
+    if (Wg->out != Wu->out || Wg->in != Wu->in) return GQ4_ERR_SHAPE;
+    if (!x || !h) return GQ4_ERR_NULL;
+    if (xdt != GQ4_F32 && xdt != GQ4_BF16) return GQ4_ERR_UNSUPPORTED;
+    if (n_tok < 1 || n_tok > (1 << 20)) return GQ4_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(h)) return GQ4_ERR_ALIGN;
+    const size_t esz = xdt == GQ4_F32 ? 4 : 2;
+    const Range hr = rng(h, (size_t)n_tok * Wg->out * esz);
+    if (overlap(hr, rng(x, (size_t)n_tok * Wg->in * esz)) ||
+        overlap(hr, rng(Wg->w, tensor_w_bytes(Wg))) || overlap(hr, rng(Wg->s, tensor_s_bytes(Wg))) ||
+        overlap(hr, rng(Wu->w, tensor_w_bytes(Wu))) || overlap(hr, rng(Wu->s, tensor_s_bytes(Wu))))
+        return GQ4_ERR_ALIAS;
+    SkinnyParams p{};
+    p.w0 = Wg->w; p.s0 = Wg->s; p.w1 = Wu->w; p.s1 = Wu->s;
+    p.O = (int)Wg->out; p.I = (int)Wg->in; p.ng = Wg->ng;
+    p.row_tiles = (int)((Wg->out + 15) / 16);
+    p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
+    p.h = h;
+    const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    return launch_skinny<kGateUp>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
+}
+
+gq4_status gq4_route(const float *logits, int64_t T, int32_t E, int32_t K, int32_t *idx,
+                     float *wts, int32_t *status, gq4_stream_t stream) {
+    if (!logits || !idx || !wts || !status) return GQ4_ERR_NULL;
+    if (T < 1 || T > (1 << 24) || E < 1 || E > kMaxExperts || K < 1 || K > E) return GQ4_ERR_SHAPE;
+    if (!aligned16(logits) || !aligned16(idx) || !aligned16(wts) || !aligned16(status)) return GQ4_ERR_ALIGN;
+    const Range lr = rng(logits, (size_t)T * E * 4);
+    const Range ir = rng(idx, (size_t)T * K * 4), wr = rng(wts, (size_t)T * K * 4), sr = rng(status, 4);
+    if (overlap(lr, ir) || overlap(lr, wr) || overlap(lr, sr) || overlap(ir, wr) || overlap(ir, sr) ||
+        overlap(wr, sr))
+        return GQ4_ERR_ALIAS;
+    return launch_route(logits, (int)T, E, K, idx, wts, status, S(stream));
+}
+
+size_t gq4_rowmap_scratch_bytes(int64_t T, int32_t K, int32_t E) {
+    if (T < 1 || K < 1 || E < 1) return 0;
+    const size_t n = (size_t)T * K;
+    return al256(16) + ((n + kChunk - 1) / kChunk) * (size_t)E * 4;
+}
+
+gq4_status gq4_rowmap(const int32_t *idx, int64_t T, int32_t K, int32_t E, int32_t *cnt,
+                      int32_t *offs, int32_t *row_tok, int32_t *row_slot, int32_t *slot_row,
+                      int32_t *n_active, int32_t *active, void *scratch, size_t scratch_bytes,
+                      gq4_stream_t stream) {
+    if (!idx || !cnt || !offs || !row_tok || !row_slot || !slot_row || !n_active || !active || !scratch)
+        return GQ4_ERR_NULL;
+    if (T < 1 || E < 1 || E > kMaxExperts || K < 1 || K > E || T * (int64_t)K > (1 << 26))
+        return GQ4_ERR_SHAPE;
+    if (scratch_bytes < gq4_rowmap_scratch_bytes(T, K, E)) return GQ4_ERR_WORKSPACE;
+    const void *ptrs[] = {idx, cnt, offs, row_tok, row_slot, slot_row, n_active, active, scratch};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return GQ4_ERR_ALIGN;
+    const size_t n = (size_t)T * K;
+    const Range rs[] = {rng(idx, n * 4), rng(cnt, E * 4), rng(offs, (E + 1) * 4), rng(row_tok, n * 4),
+                        rng(row_slot, n * 4), rng(slot_row, n * 4), rng(n_active, 4),
+                        rng(active, E * 4), rng(scratch, scratch_bytes)};
+    for (int i = 0; i < 9; ++i)
+        for (int j = i + 1; j < 9; ++j)
+            if (overlap(rs[i], rs[j])) return GQ4_ERR_ALIAS;
+    cudaStream_t s = S(stream);
+    int32_t *status = (int32_t *)scratch;
+    int32_t *chunk = (int32_t *)((char *)scratch + al256(16));
+    if (cudaMemsetAsync(status, 0, 16, s) != cudaSuccess) return GQ4_ERR_CUDA;
+    return launch_rowmap(idx, (int)n, K, E, cnt, offs, row_tok, row_slot, slot_row, n_active,
+                         active, chunk, status, s);
+}
+
+size_t moe_expert_ffn_workspace_bytes(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F) {
+    if (T < 1 || E < 1 || K < 1 || H < 1 || F < 1) return 0;
+    return moe_layout(T, E, K, H, F).total;
+}
+
+gq4_status moe_expert_ffn_routing(void *ws, size_t ws_bytes, int64_t T, int32_t E, int32_t K,
+                                  int64_t H, int64_t F, gq4_routing *out) {
+    if (!ws || !out) return GQ4_ERR_NULL;
+    if (T < 1 || E < 1 || K < 1 || K > E || H < 1 || F < 1) return GQ4_ERR_SHAPE;
+    const MoeLayout L = moe_layout(T, E, K, H, F);
+    if (ws_bytes < L.total) return GQ4_ERR_WORKSPACE;
+    out->idx = at<int32_t>(ws, L.idx);
+    out->wts = at<float>(ws, L.wts);
+    out->cnt = at<int32_t>(ws, L.cnt);
+    out->offs = at<int32_t>(ws, L.offs);
+    out->row_tok = at<int32_t>(ws, L.row_tok);
+    out->row_slot = at<int32_t>(ws, L.row_slot);
+    out->slot_row = at<int32_t>(ws, L.slot_row);
+    out->n_active = at<int32_t>(ws, L.n_active);
+    out->active = at<int32_t>(ws, L.active);
+    out->status = at<int32_t>(ws, L.status);
+    return GQ4_OK;
+}
+
+gq4_status moe_expert_ffn_status(const void *ws, size_t ws_bytes, int64_t T, int32_t E, int32_t K,
+                                 int64_t H, int64_t F, gq4_stream_t stream, int32_t *status) {
+    if (!ws || !status) return GQ4_ERR_NULL;
+    if (T < 1 || E < 1 || K < 1 || H < 1 || F < 1) return GQ4_ERR_SHAPE;
+    const MoeLayout L = moe_layout(T, E, K, H, F);
+    if (ws_bytes < L.total) return GQ4_ERR_WORKSPACE;
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, (const char *)ws + L.status, 4, cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess)
+        return GQ4_ERR_CUDA;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return GQ4_ERR_CUDA;
+    *status = v;
+    return GQ4_OK;
+}
+
+gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_tensor *Wd,
+                          const float *logits, const void *x, gq4_dtype xdt, int64_t T,
+                          int32_t E, int32_t K, float *y, void *ws, size_t ws_bytes,
+                          gq4_event_t const *stage_events, gq4_stream_t stream) {
+    gq4_status st;
+    if ((st = check_tensor(Wg, 1)) != GQ4_OK) return st;
+    if ((st = check_tensor(Wu, 1)) != GQ4_OK) return st;
+    if ((st = check_tensor(Wd, 1)) != GQ4_OK) return st;
+    if (!logits || !x || !y || !ws) return GQ4_ERR_NULL;
+    if (xdt != GQ4_BF16) return GQ4_ERR_UNSUPPORTED;
+    if (T < 1 || T > (1 << 20) || E < 1 || E > kMaxExperts || K < 1 || K > E) return GQ4_ERR_SHAPE;
+    const int64_t H = Wg->in, F = Wg->out;
+    if (Wu->out != F || Wu->in != H || Wd->out != H || Wd->in != F) return GQ4_ERR_SHAPE;
+    if (Wg->n_experts < E || Wu->n_experts < E || Wd->n_experts < E) return GQ4_ERR_SHAPE;
+    if (!aligned16(logits) || !aligned16(x) || !aligned16(y) || !aligned16(ws)) return GQ4_ERR_ALIGN;
+    const MoeLayout L = moe_layout(T, E, K, H, F);
+    if (ws_bytes < L.total) return GQ4_ERR_WORKSPACE;
+    const Range yr = rng(y, (size_t)T * H * 4), wr = rng(ws, L.total);
+    const Range ins[] = {rng(logits, (size_t)T * E * 4), rng(x, (size_t)T * H * 2),
+                         rng(Wg->w, tensor_w_bytes(Wg)), rng(Wg->s, tensor_s_bytes(Wg)),
+                         rng(Wu->w, tensor_w_bytes(Wu)), rng(Wu->s, tensor_s_bytes(Wu)),
+                         rng(Wd->w, tensor_w_bytes(Wd)), rng(Wd->s, tensor_s_bytes(Wd))};
+    for (const Range &r : ins)
+        if (overlap(yr, r) || overlap(wr, r)) return GQ4_ERR_ALIAS;
+    if (overlap(yr, wr)) return GQ4_ERR_ALIAS;
+
+    cudaStream_t s = S(stream);
+    auto mark = [&](int i) {
+        if (stage_events && stage_events[i]) cudaEventRecord((cudaEvent_t)stage_events[i], s);
+    };
+    const int n = (int)(T * K);
+    mark(0);
+    if (cudaMemsetAsync(at<int32_t>(ws, L.status), 0, 16, s) != cudaSuccess) return GQ4_ERR_CUDA;
+    // router + row map
+    if (n <= kChunk) {
+        st = launch_route_rowmap_small(logits, (int)T, E, K, ws, L, s);
+    } else {
+        st = launch_route(logits, (int)T, E, K, at<int32_t>(ws, L.idx), at<float>(ws, L.wts),
+                          at<int32_t>(ws, L.status), s);
+        if (st == GQ4_OK)
+            st = launch_rowmap(at<int32_t>(ws, L.idx), n, K, E, at<int32_t>(ws, L.cnt),
+                               at<int32_t>(ws, L.offs), at<int32_t>(ws, L.row_tok),
+                               at<int32_t>(ws, L.row_slot), at<int32_t>(ws, L.slot_row),
+                               at<int32_t>(ws, L.n_active), at<int32_t>(ws, L.active),
+                               at<int32_t>(ws, L.chunk), at<int32_t>(ws, L.status), s);
+    }
+    if (st != GQ4_OK) return st;
+    mark(1);
+
+    // expert gate+up (h in row-map order) and down with the weighted scatter-add
+    SkinnyParams p{};
+    p.offs = at<int32_t>(ws, L.offs);
+    p.cnt = at<int32_t>(ws, L.cnt);
+    p.row_tok = at<int32_t>(ws, L.row_tok);
+    p.row_slot = at<int32_t>(ws, L.row_slot);
+    p.n_active = at<int32_t>(ws, L.n_active);
+    p.active = at<int32_t>(ws, L.active);
+    p.wts = at<float>(ws, L.wts);
+    const int max_active = (int)std::min<int64_t>(E, (int64_t)T * K);
+    const int max_cols = (int)std::min<int64_t>(T, 1 << 20);
+
+    SkinnyParams pg = p;
+    pg.w0 = Wg->w; pg.s0 = Wg->s; pg.w1 = Wu->w; pg.s1 = Wu->s;
+    pg.estride_w = Wg->expert_stride_w; pg.estride_s = Wg->expert_stride_s;
+    if (Wu->expert_stride_w != Wg->expert_stride_w || Wu->expert_stride_s != Wg->expert_stride_s)
+        return GQ4_ERR_SHAPE;
+    pg.O = (int)F; pg.I = (int)H; pg.ng = Wg->ng;
+    pg.row_tiles = (int)((F + 15) / 16);
+    pg.x = x; pg.xdt = 1; pg.n_tok = (int)T;
+    pg.h = at<void>(ws, L.h);
+    pg.zero_ptr = y; pg.zero_n = T * H;
+    if ((T * H) % 4) return GQ4_ERR_SHAPE;
+    st = launch_skinny<kMoeGateUp>(pg, max_cols, false, max_active * pg.row_tiles, s);
+    if (st != GQ4_OK) return st;
+    mark(2);
+
+    SkinnyParams pd = p;
+    pd.w0 = Wd->w; pd.s0 = Wd->s;
+    pd.estride_w = Wd->expert_stride_w; pd.estride_s = Wd->expert_stride_s;
+    pd.O = (int)H; pd.I = (int)F; pd.ng = Wd->ng;
+    pd.row_tiles = (int)((H + 15) / 16);
+    pd.x = at<void>(ws, L.h); pd.xdt = 1; pd.n_tok = (int)T;
+    pd.y = y;
+    st = launch_skinny<kMoeDown>(pd, max_cols, false, max_active * pd.row_tiles, s);
+    mark(3);
+    return st;
+}
+
+}  // extern "C"

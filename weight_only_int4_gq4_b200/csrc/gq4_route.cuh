@@ -1,0 +1,243 @@
+// gq4_route.cuh -- router top-K and the on-device token -> expert row map.
+//
+// Router (colibri PR #298, "implementation complete but blocked": router top-K with a
+// taken-flag array, K passes): per token, K passes each take the largest logit among the
+// experts not yet taken; among equal logits the lower index wins.  Weights: softmax over
+// all E renormalised over the K chosen, i.e. exp(l_j - l_max) / sum_sel exp(l - l_max).
+// One warp per token; lane i holds experts i, i+32, ...
+//
+// Row map (pxq_llama.cpp release notes 2026-09-02, "Device-side MoE row map": histogram,
+// scan and fill on the device, bit-identical to the host table).  Rows of an expert are
+// ordered by ascending flat slot f = t*K + j.  Slots are cut into chunks of 1024:
+//   count: per chunk, a histogram of experts           -> chunk_cnt[c][e]
+//   scan : per expert, offsets of each chunk's rows     -> base[c][e], offs, active list
+//   fill : per chunk, a slot's rank among earlier slots of the same expert in the chunk
+//          (warp match + per-warp counts) added to base[c][e]
+// Every step is integer counting in a fixed order, so the table is deterministic.
+#pragma once
+#include "gq4_common.cuh"
+
+namespace gq4 {
+
+constexpr int kChunk = 1024;        // slots per row-map chunk (one per thread)
+constexpr int kMaxExperts = 1024;
+constexpr int kStatusNonFinite = 9; // GQ4_ERR_NONFINITE_LOGIT
+
+// Route one token with one warp.  EPL = experts per lane (>= ceil(E/32)).
+template <int EPL>
+__device__ __forceinline__ void route_token_warp(const float *lg, int E, int K, int32_t *idx,
+                                                 float *wts, int32_t *status) {
+    const int lane = threadIdx.x & 31;
+    float v[EPL];
+    bool bad = false;
+    #pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? lg[e] : -INFINITY;
+        if (e < E && (isnan(v[i]) || (isinf(v[i]) && v[i] > 0.f))) bad = true;
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    uint32_t taken = 0;
+    float my_v = 0.f;  // lane j < K keeps pick j
+    int my_e = 0;
+    float vmax = -INFINITY;
+    for (int j = 0; j < K; ++j) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+        #pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || v[i] > bv)) {
+                bv = v[i];
+                be = e;
+            }
+        }
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            const bool better = (be == 0x7fffffff) ||
+                                (oe != 0x7fffffff && (ov > bv || (ov == bv && oe < be)));
+            if (better) { bv = ov; be = oe; }
+        }
+        if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
+        if (j == 0) vmax = bv;
+        if (lane == j) { my_v = bv; my_e = be; }
+    }
+    if (!bad && isinf(vmax)) bad = true;  // no finite maximum
+    float p = (lane < K) ? expf(my_v - vmax) : 0.f;
+    float z = p;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane < K) {
+        if (bad) {
+            idx[lane] = lane;
+            wts[lane] = __uint_as_float(0x7fc00000u);
+        } else {
+            idx[lane] = my_e;
+            wts[lane] = p / z;
+        }
+    }
+    if (bad && lane == 0) atomicOr(status, kStatusNonFinite);
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) gq4_route_kernel(const float *logits, int T, int E, int K,
+                                                        int32_t *idx, float *wts, int32_t *status) {
+    const int tok = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (tok >= T) return;
+    route_token_warp<EPL>(logits + (int64_t)tok * E, E, K, idx + (int64_t)tok * K,
+                          wts + (int64_t)tok * K, status);
+}
+
+// ---- row map, chunked -------------------------------------------------------------
+// count: block c histograms slots [c*1024, (c+1)*1024) into chunk_cnt[c][E].
+// An index outside [0, E) is not counted and raises GQ4_ERR_SHAPE (3) in *status.
+__global__ void __launch_bounds__(1024) gq4_rowmap_count_kernel(const int32_t *idx, int n, int E,
+                                                                int32_t *chunk_cnt, int32_t *status) {
+    __shared__ int32_t h[kMaxExperts];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    const int f = blockIdx.x * kChunk + threadIdx.x;
+    if (f < n) {
+        const int e = idx[f];
+        if (e >= 0 && e < E) atomicAdd(&h[e], 1);
+        else atomicOr(status, 3);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_cnt[(int64_t)blockIdx.x * E + e] = h[e];
+}
+
+// Block-wide exclusive scan of one value per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_excl_scan_1024(int v, int *sh /*[32]*/, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) sh[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int s = sh[lane];
+        #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        sh[lane] = s;  // inclusive per-warp totals
+    }
+    __syncthreads();
+    const int before = (warp ? sh[warp - 1] : 0) + x - v;
+    *total = sh[31];
+    __syncthreads();
+    return before;
+}
+
+// scan: one block of 1024 threads, thread e = expert e (E <= 1024).
+__global__ void __launch_bounds__(1024) gq4_rowmap_scan_kernel(int32_t *chunk_cnt /*in: counts,
+                                                               out: bases*/, int nchunks, int E,
+                                                               int32_t *cnt, int32_t *offs,
+                                                               int32_t *n_active, int32_t *active) {
+    __shared__ int sh[32];
+    const int e = threadIdx.x;
+    int total_e = 0;
+    if (e < E)
+        for (int c = 0; c < nchunks; ++c) {
+            const int v = chunk_cnt[(int64_t)c * E + e];
+            chunk_cnt[(int64_t)c * E + e] = total_e;  // rows of e in earlier chunks
+            total_e += v;
+        }
+    int tot;
+    const int off = block_excl_scan_1024(e < E ? total_e : 0, sh, &tot);
+    const int act_before = block_excl_scan_1024((e < E && total_e > 0) ? 1 : 0, sh, &tot);
+    if (e < E) {
+        cnt[e] = total_e;
+        offs[e] = off;
+        if (total_e > 0) active[act_before] = e;
+        for (int c = 0; c < nchunks; ++c) chunk_cnt[(int64_t)c * E + e] += off;
+    }
+    if (e == 0) {
+        *n_active = tot;
+    }
+    if (e == E - 1) offs[E] = off + total_e;
+}
+
+// Rank of each slot of one chunk among the earlier slots of the same expert in the
+// chunk: per-warp counts (warp match) in shared memory wcnt[32][E], then a prefix over
+// the earlier warps.  `base` gives the first row of expert e for this chunk.  Called by
+// all 1024 threads; thread i owns slot f = chunk_start + i (e < 0: no slot).
+__device__ __forceinline__ void rowmap_fill_chunk(int f, int e, int K, int E, int32_t *wcnt,
+                                                  const int32_t *base, int32_t *row_tok,
+                                                  int32_t *row_slot, int32_t *slot_row) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(peers) - 1;
+    if (e >= 0 && lane == leader) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    if (e >= 0) {
+        int r = base[e] + __popc(peers & ((1u << lane) - 1u));
+        for (int w = 0; w < warp; ++w) r += wcnt[w * E + e];
+        row_slot[r] = f;
+        row_tok[r] = f / K;
+        slot_row[f] = r;
+    }
+}
+
+// fill: block c writes the rows of slots [c*1024, (c+1)*1024).  Dynamic shared memory:
+// 32*E ints.
+__global__ void __launch_bounds__(1024) gq4_rowmap_fill_kernel(const int32_t *idx, int n, int K, int E,
+                                                               const int32_t *base /*[nchunks][E]*/,
+                                                               int32_t *row_tok, int32_t *row_slot,
+                                                               int32_t *slot_row) {
+    extern __shared__ int32_t wcnt_dyn[];
+    const int f = blockIdx.x * kChunk + threadIdx.x;
+    int e = f < n ? idx[f] : -1;
+    if (e >= E) e = -1;
+    rowmap_fill_chunk(f, e, K, E, wcnt_dyn, base + (int64_t)blockIdx.x * E, row_tok, row_slot,
+                      slot_row);
+}
+
+// Decode path: router and the whole row map in one block of 1024 threads (T*K <= 1024).
+// Dynamic shared memory: (32 + 1) * E ints.
+template <int EPL>
+__global__ void __launch_bounds__(1024) gq4_route_rowmap_small_kernel(
+    const float *logits, int T, int E, int K, int32_t *idx, float *wts, int32_t *status,
+    int32_t *cnt, int32_t *offs, int32_t *n_active, int32_t *active, int32_t *row_tok,
+    int32_t *row_slot, int32_t *slot_row) {
+    extern __shared__ int32_t sm_dyn[];
+    int32_t *hist = sm_dyn;        // [E] counts, then offsets
+    int32_t *wcnt = sm_dyn + E;    // [32][E]
+    __shared__ int sh[32];
+    const int warp = threadIdx.x >> 5;
+    for (int t = warp; t < T; t += 32)
+        route_token_warp<EPL>(logits + (int64_t)t * E, E, K, idx + (int64_t)t * K,
+                              wts + (int64_t)t * K, status);
+    for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();  // idx written by this block is visible to the block from here
+    const int n = T * K;
+    const int f = threadIdx.x;
+    const int e = f < n ? idx[f] : -1;
+    if (e >= 0) atomicAdd(&hist[e], 1);
+    __syncthreads();
+    const int ex = threadIdx.x;
+    const int c = ex < E ? hist[ex] : 0;
+    int tot;
+    const int off = block_excl_scan_1024(c, sh, &tot);
+    const int act_before = block_excl_scan_1024((ex < E && c > 0) ? 1 : 0, sh, &tot);
+    if (ex < E) {
+        cnt[ex] = c;
+        offs[ex] = off;
+        if (c > 0) active[act_before] = ex;
+        hist[ex] = off;  // now the first row of each expert
+    }
+    if (ex == 0) *n_active = tot;
+    if (ex == E - 1) offs[E] = off + c;
+    __syncthreads();
+    rowmap_fill_chunk(f, e, K, E, wcnt, hist, row_tok, row_slot, slot_row);
+}
+
+}  // namespace gq4

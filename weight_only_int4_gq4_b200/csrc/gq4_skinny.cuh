@@ -1,0 +1,329 @@
+// gq4_skinny.cuh -- decode-regime grouped-int4 kernels (few tokens per matrix).
+//
+// What they compute (colibri PR #298 "cuda+engine: full fmt=4 (grouped int4 gs=64)
+// support"): y[c][o] = sum_g s[o][g] * sum_{k in group g} q[o][k] * x[c][k], with
+// the per-group scale applied once per 64-wide group to an f32 partial (the maintainer's
+// advice in "data request": hoist the scale per group instead of dividing k/gs per
+// element), fp32 accumulation.
+//
+// Design (B200, HBM-bound):
+//  * Weights stay in the pages' layout, [O][I/2] bytes, low nibble first.  A warp takes
+//    a 16-row x 64-column group tile (512 B): lane (g,t) reads 8 contiguous bytes of row
+//    g and of row g+8 -- every 32-byte sector is used whole.
+//  * The dot products run on the warp tensor op m16n8k16 (bf16 in, f32 out): the
+//    nibbles become exact bf16 integers (one lop3 + one bf16x2 fma per two weights), the
+//    16 contraction slots of one op are filled in an order chosen so that a lane's own
+//    bytes are its A fragment (no shuffles); the activations are staged once in shared
+//    memory in the matching order.  The op is only the dot-product engine: the bound
+//    is HBM, and this keeps the issue slots per weight near 1.
+//  * The f32 partial of each group is scaled by s[o][g] and added to the running sum.
+//  * A CTA (8 warps) owns a 16-row tile (32 with gate+up) for all columns it serves;
+//    its warps split the groups, and the eight partial tiles are summed in shared memory
+//    in a fixed order (deterministic), then the epilogue of the mode runs.
+//  * Persistent grid over units (matrix/expert, row tile); for the MoE modes the number
+//    of units is read on the device (active experts x row tiles), so no host sync.
+#pragma once
+#include "gq4_common.cuh"
+
+namespace gq4 {
+
+enum SkinnyMode { kMatvec = 0, kGateUp = 1, kMoeGateUp = 2, kMoeDown = 3 };
+
+struct SkinnyParams {
+    const uint8_t *w0;  // matrix (or gate) packed nibbles, expert 0
+    const float *s0;
+    const uint8_t *w1;  // up (gate+up modes)
+    const float *s1;
+    int64_t estride_w;  // bytes between experts
+    int64_t estride_s;  // floats between experts
+    int O, I, ng;
+    int row_tiles;      // ceil(O/16)
+    // activations: matvec/gate-up: x [n_tok][I] (xdt); moe gate-up: x [T][I] bf16
+    // (gathered through row_tok); moe down: h [T*K][I] bf16 in row-map order
+    const void *x;
+    int xdt;            // 0 f32, 1 bf16
+    int n_tok;
+    int xcols;          // staged columns the shared-memory buffer holds
+    // outputs
+    float *y;           // matvec [n_tok][O]; moe down [T][O] (accumulated)
+    void *h;            // gate-up [n_tok][O] (xdt); moe gate-up [T*K][O] bf16
+    // MoE tables (device)
+    const int32_t *offs, *cnt, *row_tok, *row_slot, *n_active, *active;
+    const float *wts;
+    float *zero_ptr;    // moe gate-up: y zeroed here before the down kernel adds into it
+    int64_t zero_n;     // floats (multiple of 4)
+};
+
+template <int MODE>
+struct ModeTraits {
+    static constexpr int kPair = (MODE == kGateUp || MODE == kMoeGateUp) ? 2 : 1;
+    static constexpr bool kMoe = (MODE == kMoeGateUp || MODE == kMoeDown);
+};
+
+// Bytes of one staged column: the I activations as bf16 plus 16 B of padding, which
+// shifts consecutive columns by four banks (conflict-free 16-byte fragment reads).
+__host__ __device__ inline int skinny_xstride(int I) { return I * 2 + 16; }
+
+// Fragment order of 16 consecutive activations v[0..15] (eight bf16x2 words w[0..7],
+// w[i] = (v[2i], v[2i+1])): step j of the group uses (v0,v4),(v1,v5) / (v2,v6),(v3,v7) /
+// (v8,v12),(v9,v13) / (v10,v14),(v11,v15) -- the same pairing the nibble decode yields
+// for the weights (nibble i and nibble i+4 of a 32-bit word land in one bf16x2).
+__device__ __forceinline__ void frag_order16(const uint32_t (&w)[8], uint4 &o0, uint4 &o1) {
+    o0.x = __byte_perm(w[0], w[2], 0x5410);
+    o0.y = __byte_perm(w[0], w[2], 0x7632);
+    o0.z = __byte_perm(w[1], w[3], 0x5410);
+    o0.w = __byte_perm(w[1], w[3], 0x7632);
+    o1.x = __byte_perm(w[4], w[6], 0x5410);
+    o1.y = __byte_perm(w[4], w[6], 0x7632);
+    o1.z = __byte_perm(w[5], w[7], 0x5410);
+    o1.w = __byte_perm(w[5], w[7], 0x7632);
+}
+
+// Stage columns [c0, c0+nc) (nc <= xcols) of the activations into shared memory.
+template <int MODE>
+__device__ __forceinline__ void skinny_stage(const SkinnyParams &p, char *xs, int c0, int nc,
+                                             int row0) {
+    const int chunks = p.ng * 4;  // 16-activation pieces per column
+    const int xstride = skinny_xstride(p.I);
+    for (int i = threadIdx.x; i < nc * chunks; i += blockDim.x) {
+        const int cl = i / chunks;
+        const int piece = i - cl * chunks;
+        const int c = c0 + cl;
+        uint32_t w[8];
+        if (MODE == kMoeGateUp || MODE == kMoeDown || p.xdt == 1) {
+            const uint16_t *src;
+            if (MODE == kMoeGateUp)
+                src = (const uint16_t *)p.x + (int64_t)p.row_tok[row0 + c] * p.I;
+            else if (MODE == kMoeDown)
+                src = (const uint16_t *)p.x + (int64_t)(row0 + c) * p.I;
+            else
+                src = (const uint16_t *)p.x + (int64_t)c * p.I;
+            const uint4 a = *((const uint4 *)(src + piece * 16));
+            const uint4 b = *((const uint4 *)(src + piece * 16 + 8));
+            w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+            w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+        } else {
+            // f32 activations: column c is split `c % 3` of token c / 3, where
+            // x = hi + mid + lo with each term a bf16 (hi = rn(x), mid = rn(x - hi),
+            // lo = rn(x - hi - mid); the differences are exact in f32).
+            const int tok = c / 3, split = c - tok * 3;
+            const float4 *src = (const float4 *)((const float *)p.x + (int64_t)tok * p.I + piece * 16);
+            #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 f = src[q];
+                const float fv[4] = {f.x, f.y, f.z, f.w};
+                uint32_t hb[4];
+                #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float r = fv[e];
+                    uint32_t b = bf16_bits_rn(r);
+                    for (int s = 0; s < split; ++s) {
+                        r = r - bf16_bits_to_f32(b);
+                        b = bf16_bits_rn(r);
+                    }
+                    hb[e] = b;
+                }
+                w[q * 2 + 0] = hb[0] | (hb[1] << 16);
+                w[q * 2 + 1] = hb[2] | (hb[3] << 16);
+            }
+        }
+        uint4 o0, o1;
+        frag_order16(w, o0, o1);
+        uint4 *dst = (uint4 *)(xs + (int64_t)cl * xstride + piece * 32);
+        dst[0] = o0;
+        dst[1] = o1;
+    }
+}
+
+template <int MODE, int NT, int UG>
+__global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
+    using TR = ModeTraits<MODE>;
+    constexpr int PAIR = TR::kPair;
+    constexpr int NCOL = NT * 8;
+    extern __shared__ __align__(16) char smem[];
+    const int xstride = skinny_xstride(p.I);
+    char *xs = smem;
+    float *red = (float *)(smem + (int64_t)p.xcols * xstride);  // [8][PAIR*16][NCOL]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int rb = p.I >> 1;  // bytes per packed row
+
+    if (MODE == kMoeGateUp && p.zero_ptr) {
+        float4 *z = (float4 *)p.zero_ptr;
+        const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_n / 4;
+             i += (int64_t)gridDim.x * blockDim.x)
+            z[i] = zero;
+    }
+
+    const int n_units = TR::kMoe ? (*p.n_active) * p.row_tiles : p.row_tiles;
+    const int gb = (warp * p.ng) >> 3, ge = ((warp + 1) * p.ng) >> 3;
+    int staged_e = -1, staged_c0 = -1;
+
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        int e = 0, rt = u, row0 = 0, cols;
+        if (TR::kMoe) {
+            const int a = u / p.row_tiles;
+            rt = u - a * p.row_tiles;
+            e = p.active[a];
+            row0 = p.offs[e];
+            cols = p.cnt[e];
+        } else {
+            cols = (p.xdt == 0) ? 3 * p.n_tok : p.n_tok;
+        }
+        const uint8_t *W0 = p.w0 + (int64_t)e * p.estride_w;
+        const float *S0 = p.s0 + (int64_t)e * p.estride_s;
+        const uint8_t *W1 = PAIR == 2 ? p.w1 + (int64_t)e * p.estride_w : nullptr;
+        const float *S1 = PAIR == 2 ? p.s1 + (int64_t)e * p.estride_s : nullptr;
+        const int rA = rt * 16 + g, rB = rA + 8;
+        const bool vA = rA < p.O, vB = rB < p.O;
+
+        for (int c0 = 0; c0 < cols; c0 += p.xcols) {
+            const int nc = min(p.xcols, cols - c0);
+            if (e != staged_e || c0 != staged_c0) {
+                __syncthreads();  // previous readers of xs are done
+                skinny_stage<MODE>(p, xs, c0, nc, row0);
+                __syncthreads();
+                staged_e = e;
+                staged_c0 = c0;
+            }
+            // f32 activations use three staged columns per token: a pass holds whole tokens
+            const int pw = (!TR::kMoe && p.xdt == 0) ? (NCOL / 3) * 3 : NCOL;
+            for (int cc = 0; cc < nc; cc += pw) {
+                const int ncc = min(pw, nc - cc);
+                float acc[PAIR][NT][4];
+                #pragma unroll
+                for (int m = 0; m < PAIR; ++m)
+                    #pragma unroll
+                    for (int n = 0; n < NT; ++n)
+                        #pragma unroll
+                        for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+
+                for (int G0 = gb; G0 < ge; G0 += UG) {
+                    uint2 wa[PAIR][UG], wb[PAIR][UG];
+                    float sa[PAIR][UG], sb[PAIR][UG];
+                    #pragma unroll
+                    for (int q = 0; q < UG; ++q) {
+                        const int G = G0 + q;
+                        const bool ok = G < ge;
+                        #pragma unroll
+                        for (int m = 0; m < PAIR; ++m) {
+                            const uint8_t *Wm = m ? W1 : W0;
+                            const float *Sm = m ? S1 : S0;
+                            const int64_t off = (int64_t)G * 32 + t * 8;
+                            wa[m][q] = (ok && vA) ? ldg_stream_u2(Wm + (int64_t)rA * rb + off) : make_uint2(0, 0);
+                            wb[m][q] = (ok && vB) ? ldg_stream_u2(Wm + (int64_t)rB * rb + off) : make_uint2(0, 0);
+                            sa[m][q] = (ok && vA) ? ldg_f32(Sm + (int64_t)rA * p.ng + G) : 0.f;
+                            sb[m][q] = (ok && vB) ? ldg_f32(Sm + (int64_t)rB * p.ng + G) : 0.f;
+                        }
+                    }
+                    #pragma unroll
+                    for (int q = 0; q < UG; ++q) {
+                        const int G = G0 + q;
+                        if (G >= ge) break;
+                        // A fragments: r[2j] / r[2j+1] are the two bf16x2 pairs of step j
+                        uint32_t ra[PAIR][8], rbv[PAIR][8];
+                        #pragma unroll
+                        for (int m = 0; m < PAIR; ++m) {
+                            #pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                ra[m][i] = nib2_to_bf16x2(wa[m][q].x >> (4 * i));
+                                ra[m][4 + i] = nib2_to_bf16x2(wa[m][q].y >> (4 * i));
+                                rbv[m][i] = nib2_to_bf16x2(wb[m][q].x >> (4 * i));
+                                rbv[m][4 + i] = nib2_to_bf16x2(wb[m][q].y >> (4 * i));
+                            }
+                        }
+                        #pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            const int cl = cc + n * 8 + g;  // staged column this lane feeds
+                            uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+                            if (n * 8 + g < ncc) {
+                                const uint4 *src = (const uint4 *)(xs + (int64_t)cl * xstride + (G * 4 + t) * 32);
+                                b0 = src[0];
+                                b1 = src[1];
+                            }
+                            const uint32_t bf[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                            #pragma unroll
+                            for (int m = 0; m < PAIR; ++m) {
+                                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                                #pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const uint32_t a[4] = {ra[m][2 * j], rbv[m][2 * j], ra[m][2 * j + 1], rbv[m][2 * j + 1]};
+                                    mma_bf16_16816(d, a, bf[2 * j], bf[2 * j + 1], d);
+                                }
+                                acc[m][n][0] = fmaf(sa[m][q], d[0], acc[m][n][0]);
+                                acc[m][n][1] = fmaf(sa[m][q], d[1], acc[m][n][1]);
+                                acc[m][n][2] = fmaf(sb[m][q], d[2], acc[m][n][2]);
+                                acc[m][n][3] = fmaf(sb[m][q], d[3], acc[m][n][3]);
+                            }
+                        }
+                    }
+                }
+                // cross-warp reduction of the 8 partial tiles (fixed order)
+                #pragma unroll
+                for (int m = 0; m < PAIR; ++m)
+                    #pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        float *r0 = red + ((warp * PAIR + m) * 16 + g) * NCOL + n * 8 + 2 * t;
+                        r0[0] = acc[m][n][0];
+                        r0[1] = acc[m][n][1];
+                        r0[8 * NCOL] = acc[m][n][2];
+                        r0[8 * NCOL + 1] = acc[m][n][3];
+                    }
+                __syncthreads();
+                if (!TR::kMoe && p.xdt == 0) {
+                    // f32 activations: three staged columns per token
+                    const int ntok = ncc / 3;
+                    for (int i = threadIdx.x; i < 16 * ntok; i += blockDim.x) {
+                        const int row = i & 15, tl = i >> 4;
+                        const int o = rt * 16 + row;
+                        if (o >= p.O) continue;
+                        const int tok = (c0 + cc) / 3 + tl;
+                        float v[PAIR];
+                        #pragma unroll
+                        for (int m = 0; m < PAIR; ++m) {
+                            float s = 0.f;
+                            for (int sp = 0; sp < 3; ++sp)
+                                for (int w = 0; w < 8; ++w)
+                                    s += red[((w * PAIR + m) * 16 + row) * NCOL + tl * 3 + sp];
+                            v[m] = s;
+                        }
+                        if (MODE == kMatvec)
+                            p.y[(int64_t)tok * p.O + o] = v[0];
+                        else
+                            ((float *)p.h)[(int64_t)tok * p.O + o] = silu_mul(v[0], v[PAIR - 1]);
+                    }
+                } else {
+                    for (int i = threadIdx.x; i < 16 * ncc; i += blockDim.x) {
+                        const int row = i & 15, cl = i >> 4;
+                        const int o = rt * 16 + row;
+                        if (o >= p.O) continue;
+                        float v[PAIR];
+                        #pragma unroll
+                        for (int m = 0; m < PAIR; ++m) {
+                            float s = 0.f;
+                            for (int w = 0; w < 8; ++w) s += red[((w * PAIR + m) * 16 + row) * NCOL + cl];
+                            v[m] = s;
+                        }
+                        const int c = c0 + cc + cl;
+                        if (MODE == kMatvec) {
+                            p.y[(int64_t)c * p.O + o] = v[0];
+                        } else if (MODE == kGateUp) {
+                            ((uint16_t *)p.h)[(int64_t)c * p.O + o] = (uint16_t)bf16_bits_rn(silu_mul(v[0], v[1]));
+                        } else if (MODE == kMoeGateUp) {
+                            ((uint16_t *)p.h)[(int64_t)(row0 + c) * p.O + o] = (uint16_t)bf16_bits_rn(silu_mul(v[0], v[1]));
+                        } else {  // kMoeDown: weighted scatter-add into y
+                            const int r = row0 + c;
+                            const float wt = p.wts[p.row_slot[r]];
+                            atomicAdd(p.y + (int64_t)p.row_tok[r] * p.O + o, wt * v[0]);
+                        }
+                    }
+                }
+                __syncthreads();  // red is rewritten by the next pass
+            }
+        }
+    }
+}
+
+}  // namespace gq4
