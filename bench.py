@@ -235,6 +235,9 @@ def main():
 
     # ---- device-timed steps (L2 flushed between steps, outside the events)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for row in evs:  # torch creates the CUDA event lazily, at its first record
+        for e in row:
+            e.record(stream)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

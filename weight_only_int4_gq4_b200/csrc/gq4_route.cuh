@@ -38,8 +38,10 @@ __device__ __forceinline__ void route_token_warp(const float *lg, int E, int K, 
     }
     bad = __any_sync(0xffffffffu, bad);
     uint32_t taken = 0;
-    float my_v = 0.f;  // lane j < K keeps pick j
-    int my_e = 0;
+    float my_v[EPL];  // pick j is kept by lane j % 32 in slot j / 32 (K <= E <= 32*EPL)
+    int my_e[EPL];
+    #pragma unroll
+    for (int i = 0; i < EPL; ++i) { my_v[i] = -INFINITY; my_e[i] = 0; }
     float vmax = -INFINITY;
     for (int j = 0; j < K; ++j) {
         float bv = -INFINITY;
@@ -62,20 +64,33 @@ __device__ __forceinline__ void route_token_warp(const float *lg, int E, int K, 
         }
         if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
         if (j == 0) vmax = bv;
-        if (lane == j) { my_v = bv; my_e = be; }
+        if ((j & 31) == lane) {
+            #pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (i == (j >> 5)) { my_v[i] = bv; my_e[i] = be; }
+        }
     }
     if (!bad && isinf(vmax)) bad = true;  // no finite maximum
-    float p = (lane < K) ? expf(my_v - vmax) : 0.f;
-    float z = p;
+    float p[EPL];
+    float z = 0.f;
+    #pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        p[i] = (lane + 32 * i < K) ? expf(my_v[i] - vmax) : 0.f;
+        z += p[i];
+    }
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane < K) {
-        if (bad) {
-            idx[lane] = lane;
-            wts[lane] = __uint_as_float(0x7fc00000u);
-        } else {
-            idx[lane] = my_e;
-            wts[lane] = p / z;
+    #pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int j = lane + 32 * i;
+        if (j < K) {
+            if (bad) {
+                idx[j] = j;
+                wts[j] = __uint_as_float(0x7fc00000u);
+            } else {
+                idx[j] = my_e[i];
+                wts[j] = p[i] / z;
+            }
         }
     }
     if (bad && lane == 0) atomicOr(status, kStatusNonFinite);
