@@ -10,6 +10,10 @@
  *     converted by XOR 0x88 per byte at upload);
  *   - one f32 scale per `gs` consecutive inputs of each row: scales[o*ng + k/gs] with
  *     ng = ceil(in/gs), so w[o][k] = scales[o*ng + k/gs] * q[o][k].
+ * Device layout: rows and scales as above; inside every 32-bit word (the 8 weights
+ * k = 8i..8i+7 of a row) the nibbles are reordered to k0,k2,k4,k6 in bits 0-15 and
+ * k1,k3,k5,k7 in bits 16-31 (each group ascending from the low bits).  gq4_upload
+ * writes this order; gq4_tensor_init expects data already in it.
  *
  * Conventions shared by every call:
  *   - The caller owns all memory.  Device buffers are passed as raw device pointers and
@@ -110,9 +114,10 @@ gq4_status gq4_device_bytes(int64_t out, int64_t in, int32_t gs, int32_t n_exper
                             size_t *w_bytes, size_t *s_bytes);
 
 /* Copy packed weights and scales of n_experts matrices from host memory into
- * caller-owned device buffers and fill *desc (expert strides = the tight sizes).  With
- * src_offset_binary = 1 each byte is XORed with 0x88 on the device after the copy
- * (offset_to_signed_s4).  Asynchronous on `stream`; the host buffers must stay valid
+ * caller-owned device buffers, reorder the nibbles of each 32-bit word into the device
+ * layout (on the device), and fill *desc (expert strides = the tight sizes).  With
+ * src_offset_binary = 1 each byte is XORed with 0x88 first (offset_to_signed_s4).
+ * `in` must be a multiple of 8 (GQ4_ERR_UNSUPPORTED otherwise).  Asynchronous on `stream`; the host buffers must stay valid
  * until the stream reaches this point.  Device buffers must be at least the sizes from
  * gq4_device_bytes and 16-byte aligned. */
 gq4_status gq4_upload(const uint8_t *packed_host, const float *scales_host, int64_t out,

@@ -17,6 +17,20 @@ if torch.cuda.is_available():
     from weight_only_int4_gq4_b200 import gq4
 
 
+def device_words_to_host(dev: np.ndarray) -> np.ndarray:
+    """Undo the device nibble order (even-k nibbles in the low half-word, odd-k in the
+    high half-word of each 32-bit word) to get the pages' low-nibble-first bytes."""
+    w = dev.reshape(dev.shape[0], -1).view(np.uint32)
+    nib = np.stack([(w >> (4 * i)) & 15 for i in range(8)], -1)  # slots 0..7
+    k = np.empty_like(nib)
+    k[..., 0::2] = nib[..., 0:4]
+    k[..., 1::2] = nib[..., 4:8]
+    host = np.zeros_like(w)
+    for i in range(8):
+        host |= (k[..., i] << (4 * i)).astype(np.uint32)
+    return host.view(np.uint8).reshape(dev.shape)
+
+
 def _x_torch(x):
     return bf16_to_torch(x) if x.dtype == np.uint16 else torch.from_numpy(x).cuda()
 
@@ -60,7 +74,7 @@ def test_matvec_offset_binary_upload():
     pob = oracle.pack(q, offset_binary=True)           # host file in offset binary
     assert np.array_equal(gq4.pack(u, offset_binary=True), oracle.pack(q))
     W = gq4.upload(pob, s, offset_binary=True)         # XOR 0x88 on the device
-    assert np.array_equal(W.w.cpu().numpy().reshape(O, I // 2), oracle.pack(q))
+    assert np.array_equal(device_words_to_host(W.w.cpu().numpy().reshape(O, I // 2)), oracle.pack(q))
     x = synth.x_normal(5, 1, I, "bf16")
     check_close(gq4.matvec(W, bf16_to_torch(x)).cpu().numpy(), *oracle.matvec(oracle.pack(q), s, x))
 
@@ -224,7 +238,11 @@ def _toy(T, E, K, H=128, F=128, seed=3, **kw):
 
 @pytest.mark.parametrize("T,E,K,H,F", [(5, 4, 2, 128, 128), (1, 1, 1, 64, 64), (3, 8, 8, 192, 256),
                                        (17, 16, 4, 256, 128), (40, 32, 8, 128, 192),
-                                       (300, 16, 4, 128, 64)])
+                                       (300, 16, 4, 128, 64),
+                                       # tensor-core path (experts with >= 24 rows), mixed with
+                                       # the decode path, multi-pass experts (> 192 rows)
+                                       (64, 4, 2, 256, 128), (40, 8, 4, 384, 192), (300, 2, 1, 128, 64),
+                                       (500, 2, 2, 128, 128), (48, 4, 2, 192, 128), (130, 6, 3, 512, 256)])
 def test_moe_small_full_oracle(T, E, K, H, F):
     s = MoESet(_toy(T, E, K, H, F))
     y, ws = s.run()

@@ -1,7 +1,7 @@
 // gq4_host.cu -- the C ABI of libgq4 (declared in include/gq4.h): argument checks,
 // workspace layout and kernel launches.  Every compute step runs in the kernels of
-// gq4_skinny.cuh / gq4_route.cuh / gq4_prefill.cuh; this file only validates and
-// launches.
+// gq4_skinny.cuh / gq4_route.cuh / gq4_tc.cuh; this file only validates, lays out the
+// workspace, encodes TMA descriptors and launches.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -13,6 +13,7 @@
 #include "gq4_common.cuh"
 #include "gq4_route.cuh"
 #include "gq4_skinny.cuh"
+#include "gq4_tc.cuh"
 
 using namespace gq4;
 
@@ -116,13 +117,16 @@ gq4_status launch_skinny(SkinnyParams p, int max_cols, bool f32x, int units_uppe
 // ---- MoE workspace layout --------------------------------------------------------------
 struct MoeLayout {
     size_t status, idx, wts, cnt, offs, row_tok, row_slot, slot_row, n_active, active, chunk,
-        h, total;
+        h, lists, xg, total;
 };
+
+// Experts with at least this many rows go to the tensor-core (tcgen05) kernels, the
+// others to the decode kernels.
+constexpr int kLargeMin = 24;
 
 inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 MoeLayout moe_layout(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F) {
-    (void)H;
     MoeLayout L{};
     const size_t n = (size_t)T * K;
     const size_t nchunks = (n + kChunk - 1) / kChunk;
@@ -139,12 +143,19 @@ MoeLayout moe_layout(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F) {
     L.active = o; o = al256(o + (size_t)E * 4);
     L.chunk = o; o = al256(o + nchunks * (size_t)E * 4);
     L.h = o; o = al256(o + n * (size_t)F * 2);
+    L.lists = o; o = al256(o + (size_t)(2 * E + 8) * 4);  // n_small, n_large, small[E], large[E]
+    L.xg = o; o = al256(o + (T >= kLargeMin ? n * (size_t)H * 2 : 0));
     L.total = o;
     return L;
 }
 
 template <typename T>
 inline T *at(void *ws, size_t off) { return reinterpret_cast<T *>((char *)ws + off); }
+
+ExpertLists moe_lists(void *ws, const MoeLayout &L, int E, int thr) {
+    int32_t *b = at<int32_t>(ws, L.lists);
+    return ExpertLists{b, b + 8, b + 1, b + 8 + E, thr};
+}
 
 int epl_for(int E) {
     int epl = 1;
@@ -166,10 +177,11 @@ gq4_status launch_route(const float *logits, int T, int E, int K, int32_t *idx, 
 
 gq4_status launch_rowmap(const int32_t *idx, int n, int K, int E, int32_t *cnt, int32_t *offs,
                          int32_t *row_tok, int32_t *row_slot, int32_t *slot_row, int32_t *n_active,
-                         int32_t *active, int32_t *chunk, int32_t *status, cudaStream_t st) {
+                         int32_t *active, int32_t *chunk, int32_t *status, ExpertLists lists,
+                         cudaStream_t st) {
     const int nchunks = (n + kChunk - 1) / kChunk;
     gq4_rowmap_count_kernel<<<nchunks, kChunk, 0, st>>>(idx, n, E, chunk, status);
-    gq4_rowmap_scan_kernel<<<1, 1024, 0, st>>>(chunk, nchunks, E, cnt, offs, n_active, active);
+    gq4_rowmap_scan_kernel<<<1, 1024, 0, st>>>(chunk, nchunks, E, cnt, offs, n_active, active, lists);
     const size_t smem = (size_t)32 * E * 4;
     if (allow_smem(gq4_rowmap_fill_kernel, smem) != cudaSuccess) return GQ4_ERR_CUDA;
     gq4_rowmap_fill_kernel<<<nchunks, kChunk, smem, st>>>(idx, n, K, E, chunk, row_tok, row_slot,
@@ -178,13 +190,13 @@ gq4_status launch_rowmap(const int32_t *idx, int n, int K, int E, int32_t *cnt, 
 }
 
 gq4_status launch_route_rowmap_small(const float *logits, int T, int E, int K, void *ws,
-                                     const MoeLayout &L, cudaStream_t st) {
+                                     const MoeLayout &L, ExpertLists lists, cudaStream_t st) {
     const size_t smem = (size_t)33 * E * 4;
     int32_t *status = at<int32_t>(ws, L.status);
 #define SMALL_ARGS logits, T, E, K, at<int32_t>(ws, L.idx), at<float>(ws, L.wts), status,      \
                    at<int32_t>(ws, L.cnt), at<int32_t>(ws, L.offs), at<int32_t>(ws, L.n_active), \
                    at<int32_t>(ws, L.active), at<int32_t>(ws, L.row_tok),                        \
-                   at<int32_t>(ws, L.row_slot), at<int32_t>(ws, L.slot_row)
+                   at<int32_t>(ws, L.row_slot), at<int32_t>(ws, L.slot_row), lists
     switch (epl_for(E)) {
 #define SMALL_CASE(N)                                                                    \
     case N:                                                                              \
@@ -199,14 +211,66 @@ gq4_status launch_route_rowmap_small(const float *logits, int T, int E, int K, v
     return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
 }
 
-__global__ void gq4_xor88_kernel(uint4 *p, size_t n16, uint8_t *tail, size_t ntail) {
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n16) {
-        uint4 v = p[i];
-        v.x ^= 0x88888888u; v.y ^= 0x88888888u; v.z ^= 0x88888888u; v.w ^= 0x88888888u;
-        p[i] = v;
+// Upload repack: host rows hold the weights of k = 8i..8i+7 in one little-endian 32-bit
+// word as nibbles k0..k7 (low nibble first).  The device word holds the even-k nibbles
+// (k0,k2,k4,k6) in its low 16 bits and the odd-k nibbles (k1,k3,k5,k7) in its high 16
+// bits, so one lop3 turns nibble slots i and i+4 into the bf16 pair (k_2i, k_2i+1) of
+// consecutive columns.  With offset-binary input every nibble's top bit is flipped
+// first (XOR 0x88 per byte).
+__device__ __forceinline__ uint32_t compact_nibbles(uint32_t v) {  // nibbles at bits 0,8,16,24
+    v = (v | (v >> 4)) & 0x00FF00FFu;
+    return (v | (v >> 8)) & 0x0000FFFFu;
+}
+
+__global__ void gq4_repack_kernel(uint32_t *w, size_t nwords, uint32_t flip) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nwords;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const uint32_t v = w[i] ^ flip;
+        w[i] = compact_nibbles(v & 0x0F0F0F0Fu) | (compact_nibbles((v >> 4) & 0x0F0F0F0Fu) << 16);
     }
-    if (i < ntail) tail[i] ^= 0x88u;
+}
+
+// ---- TMA descriptors (driver entry point, no libcuda link) ------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    });
+    return fn;
+}
+
+// 2-D map over a row-major [rows][cols] array; box = box_cols x box_rows.
+bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t esz, uint64_t cols,
+                  uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * esz};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+gq4_status launch_tc(const CUtensorMap &w0, const CUtensorMap &w1, const CUtensorMap &x,
+                     const TcParams &p, int units_upper, cudaStream_t st) {
+    auto kern = gq4_tc_kernel<MODE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes) != cudaSuccess)
+        return GQ4_ERR_CUDA;
+    const int grid = std::max(1, std::min(units_upper, sm_count()));
+    kern<<<grid, kTcThreads, kTcSmemBytes, st>>>(w0, w1, x, p);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
 }
 
 }  // namespace
@@ -291,16 +355,17 @@ gq4_status gq4_upload(const uint8_t *packed_host, const float *scales_host, int6
     gq4_status st = gq4_device_bytes(out, in, gs, n_experts, &wb, &sb);
     if (st != GQ4_OK) return st;
     if (d_w_bytes < wb || d_s_bytes < sb) return GQ4_ERR_SHAPE;
+    if (in % 8) return GQ4_ERR_UNSUPPORTED;  // device words hold 8 weights of one row
     if (!aligned16(d_w) || !aligned16(d_s)) return GQ4_ERR_ALIGN;
     if (overlap(rng(d_w, wb), rng(d_s, sb))) return GQ4_ERR_ALIAS;
     cudaStream_t s = S(stream);
     if (cudaMemcpyAsync(d_w, packed_host, wb, cudaMemcpyHostToDevice, s) != cudaSuccess) return GQ4_ERR_CUDA;
     if (cudaMemcpyAsync(d_s, scales_host, sb, cudaMemcpyHostToDevice, s) != cudaSuccess) return GQ4_ERR_CUDA;
-    if (src_offset_binary) {
-        const size_t n16 = wb / 16, ntail = wb % 16;
-        const size_t nthreads = std::max(n16, ntail);
-        const unsigned grid = (unsigned)((nthreads + 255) / 256);
-        if (grid) gq4_xor88_kernel<<<grid, 256, 0, s>>>((uint4 *)d_w, n16, (uint8_t *)d_w + n16 * 16, ntail);
+    {
+        const size_t nwords = wb / 4;
+        const unsigned grid = (unsigned)std::min<size_t>((nwords + 255) / 256, (size_t)sm_count() * 8);
+        gq4_repack_kernel<<<std::max(grid, 1u), 256, 0, s>>>((uint32_t *)d_w, nwords,
+                                                           src_offset_binary ? 0x88888888u : 0u);
         if (cudaGetLastError() != cudaSuccess) return GQ4_ERR_CUDA;
     }
     return gq4_tensor_init(d_w, d_s, out, in, gs, n_experts, desc);
@@ -399,7 +464,7 @@ gq4_status gq4_rowmap(const int32_t *idx, int64_t T, int32_t K, int32_t E, int32
     int32_t *chunk = (int32_t *)((char *)scratch + al256(16));
     if (cudaMemsetAsync(status, 0, 16, s) != cudaSuccess) return GQ4_ERR_CUDA;
     return launch_rowmap(idx, (int)n, K, E, cnt, offs, row_tok, row_slot, slot_row, n_active,
-                         active, chunk, status, s);
+                         active, chunk, status, ExpertLists{nullptr, nullptr, nullptr, nullptr, 1 << 30}, s);
 }
 
 size_t moe_expert_ffn_workspace_bytes(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F) {
@@ -473,9 +538,15 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     const int n = (int)(T * K);
     mark(0);
     if (cudaMemsetAsync(at<int32_t>(ws, L.status), 0, 16, s) != cudaSuccess) return GQ4_ERR_CUDA;
+    // an expert can reach kLargeMin rows only if T does; the tensor-core kernels tile the
+    // down rows by 128 and load scales four groups at a time
+    const bool tc = T >= kLargeMin && H % 128 == 0 && F % 64 == 0 && Wg->ng % 4 == 0 && Wd->ng % 4 == 0 &&
+                    Wg->expert_stride_w % (H / 2) == 0 && Wu->expert_stride_w == Wg->expert_stride_w &&
+                    Wd->expert_stride_w % (F / 2) == 0;
+    const ExpertLists lists = moe_lists(ws, L, E, tc ? kLargeMin : (1 << 30));
     // router + row map
     if (n <= kChunk) {
-        st = launch_route_rowmap_small(logits, (int)T, E, K, ws, L, s);
+        st = launch_route_rowmap_small(logits, (int)T, E, K, ws, L, lists, s);
     } else {
         st = launch_route(logits, (int)T, E, K, at<int32_t>(ws, L.idx), at<float>(ws, L.wts),
                           at<int32_t>(ws, L.status), s);
@@ -484,7 +555,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
                                at<int32_t>(ws, L.offs), at<int32_t>(ws, L.row_tok),
                                at<int32_t>(ws, L.row_slot), at<int32_t>(ws, L.slot_row),
                                at<int32_t>(ws, L.n_active), at<int32_t>(ws, L.active),
-                               at<int32_t>(ws, L.chunk), at<int32_t>(ws, L.status), s);
+                               at<int32_t>(ws, L.chunk), at<int32_t>(ws, L.status), lists, s);
     }
     if (st != GQ4_OK) return st;
     mark(1);
@@ -495,8 +566,8 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     p.cnt = at<int32_t>(ws, L.cnt);
     p.row_tok = at<int32_t>(ws, L.row_tok);
     p.row_slot = at<int32_t>(ws, L.row_slot);
-    p.n_active = at<int32_t>(ws, L.n_active);
-    p.active = at<int32_t>(ws, L.active);
+    p.n_active = lists.n_small;  // the decode kernels take the experts with few rows
+    p.active = lists.small;
     p.wts = at<float>(ws, L.wts);
     const int max_active = (int)std::min<int64_t>(E, (int64_t)T * K);
     const int max_cols = (int)std::min<int64_t>(T, 1 << 20);
@@ -512,8 +583,44 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     pg.h = at<void>(ws, L.h);
     pg.zero_ptr = y; pg.zero_n = T * H;
     if ((T * H) % 4) return GQ4_ERR_SHAPE;
-    st = launch_skinny<kMoeGateUp>(pg, max_cols, false, max_active * pg.row_tiles, s);
+    const int small_cols = (int)std::min<int64_t>(max_cols, tc ? kLargeMin - 1 : max_cols);
+    st = launch_skinny<kMoeGateUp>(pg, small_cols, false, max_active * pg.row_tiles, s);
     if (st != GQ4_OK) return st;
+
+    // experts with many rows: gathered activations, tensor-core gate+up and down
+    CUtensorMap tm_g, tm_u, tm_d, tm_x, tm_h;
+    TcParams tp{};
+    if (tc) {
+        const int max_large = std::max(1, std::min<int>(E, (int)(T * K / kLargeMin)));
+        const int chunks = (int)(H / 8);
+        gq4_gather_rows_kernel<<<sm_count() * 8, 256, 0, s>>>((const uint4 *)x, at<int32_t>(ws, L.row_tok),
+                                                             n, chunks, at<uint4>(ws, L.xg));
+        if (cudaGetLastError() != cudaSuccess) return GQ4_ERR_CUDA;
+        const uint64_t rows_gu = (uint64_t)(Wg->n_experts - 1) * (Wg->expert_stride_w / (H / 2)) + F;
+        const uint64_t rows_d = (uint64_t)(Wd->n_experts - 1) * (Wd->expert_stride_w / (F / 2)) + H;
+        if (!make_tmap_2d(&tm_g, Wg->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H / 2, rows_gu, 32, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !make_tmap_2d(&tm_u, Wu->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H / 2, rows_gu, 32, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !make_tmap_2d(&tm_d, Wd->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, F / 2, rows_d, 32, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !make_tmap_2d(&tm_x, at<void>(ws, L.xg), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, n, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_2d(&tm_h, at<void>(ws, L.h), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, F, n, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+            return GQ4_ERR_CUDA;
+        tp.offs = at<int32_t>(ws, L.offs);
+        tp.cnt = at<int32_t>(ws, L.cnt);
+        tp.n_large = lists.n_large;
+        tp.large = lists.large;
+        tp.row_tok = at<int32_t>(ws, L.row_tok);
+        tp.row_slot = at<int32_t>(ws, L.row_slot);
+        tp.wts = at<float>(ws, L.wts);
+        tp.status = at<int32_t>(ws, L.status);
+        tp.h = at<uint16_t>(ws, L.h);
+        tp.y = y;
+        TcParams tg = tp;
+        tg.s0 = Wg->s; tg.s1 = Wu->s; tg.estride_s = Wg->expert_stride_s;
+        tg.O = (int)F; tg.I = (int)H; tg.ng = Wg->ng; tg.m_tiles = (int)(F / 64);
+        tg.estride_rows = (int)(Wg->expert_stride_w / (H / 2));
+        st = launch_tc<0>(tm_g, tm_u, tm_x, tg, max_large * tg.m_tiles, s);
+        if (st != GQ4_OK) return st;
+    }
     mark(2);
 
     SkinnyParams pd = p;
@@ -523,7 +630,16 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     pd.row_tiles = (int)((H + 15) / 16);
     pd.x = at<void>(ws, L.h); pd.xdt = 1; pd.n_tok = (int)T;
     pd.y = y;
-    st = launch_skinny<kMoeDown>(pd, max_cols, false, max_active * pd.row_tiles, s);
+    st = launch_skinny<kMoeDown>(pd, small_cols, false, max_active * pd.row_tiles, s);
+    if (st != GQ4_OK) return st;
+    if (tc) {
+        const int max_large = std::max(1, std::min<int>(E, (int)(T * K / kLargeMin)));
+        TcParams td = tp;
+        td.s0 = Wd->s; td.s1 = Wd->s; td.estride_s = Wd->expert_stride_s;
+        td.O = (int)H; td.I = (int)F; td.ng = Wd->ng; td.m_tiles = (int)(H / 128);
+        td.estride_rows = (int)(Wd->expert_stride_w / (F / 2));
+        st = launch_tc<1>(tm_d, tm_d, tm_h, td, max_large * td.m_tiles, s);
+    }
     mark(3);
     return st;
 }

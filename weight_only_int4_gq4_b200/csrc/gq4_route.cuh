@@ -150,11 +150,30 @@ __device__ __forceinline__ int block_excl_scan_1024(int v, int *sh /*[32]*/, int
     return before;
 }
 
+// Expert lists for the two GEMM regimes: small (0 < cnt < thr: the decode kernels) and
+// large (cnt >= thr: the tensor-core kernels), each ascending.  Null pointers: skipped.
+struct ExpertLists {
+    int32_t *n_small, *small, *n_large, *large;
+    int thr;
+};
+
+__device__ __forceinline__ void classify_experts(int e, int E, int c, int *sh, const ExpertLists &L) {
+    int tot;
+    const bool is_small = e < E && c > 0 && c < L.thr, is_large = e < E && c >= L.thr;
+    const int sb = block_excl_scan_1024(is_small ? 1 : 0, sh, &tot);
+    if (is_small && L.small) L.small[sb] = e;
+    if (e == 0 && L.n_small) *L.n_small = tot;
+    const int lb = block_excl_scan_1024(is_large ? 1 : 0, sh, &tot);
+    if (is_large && L.large) L.large[lb] = e;
+    if (e == 0 && L.n_large) *L.n_large = tot;
+}
+
 // scan: one block of 1024 threads, thread e = expert e (E <= 1024).
 __global__ void __launch_bounds__(1024) gq4_rowmap_scan_kernel(int32_t *chunk_cnt /*in: counts,
                                                                out: bases*/, int nchunks, int E,
                                                                int32_t *cnt, int32_t *offs,
-                                                               int32_t *n_active, int32_t *active) {
+                                                               int32_t *n_active, int32_t *active,
+                                                               ExpertLists lists) {
     __shared__ int sh[32];
     const int e = threadIdx.x;
     int total_e = 0;
@@ -173,10 +192,9 @@ __global__ void __launch_bounds__(1024) gq4_rowmap_scan_kernel(int32_t *chunk_cn
         if (total_e > 0) active[act_before] = e;
         for (int c = 0; c < nchunks; ++c) chunk_cnt[(int64_t)c * E + e] += off;
     }
-    if (e == 0) {
-        *n_active = tot;
-    }
+    if (e == 0) *n_active = tot;
     if (e == E - 1) offs[E] = off + total_e;
+    classify_experts(e, E, total_e, sh, lists);
 }
 
 // Rank of each slot of one chunk among the earlier slots of the same expert in the
@@ -222,7 +240,7 @@ template <int EPL>
 __global__ void __launch_bounds__(1024) gq4_route_rowmap_small_kernel(
     const float *logits, int T, int E, int K, int32_t *idx, float *wts, int32_t *status,
     int32_t *cnt, int32_t *offs, int32_t *n_active, int32_t *active, int32_t *row_tok,
-    int32_t *row_slot, int32_t *slot_row) {
+    int32_t *row_slot, int32_t *slot_row, ExpertLists lists) {
     extern __shared__ int32_t sm_dyn[];
     int32_t *hist = sm_dyn;        // [E] counts, then offsets
     int32_t *wcnt = sm_dyn + E;    // [32][E]
@@ -251,8 +269,22 @@ __global__ void __launch_bounds__(1024) gq4_route_rowmap_small_kernel(
     }
     if (ex == 0) *n_active = tot;
     if (ex == E - 1) offs[E] = off + c;
+    classify_experts(ex, E, c, sh, lists);
     __syncthreads();
     rowmap_fill_chunk(f, e, K, E, wcnt, hist, row_tok, row_slot, slot_row);
 }
 
+}  // namespace gq4
+
+namespace gq4 {
+// Gather the activation rows of the row map into row-map order: xg[r] = x[row_tok[r]].
+__global__ void gq4_gather_rows_kernel(const uint4 *x, const int32_t *row_tok, int n_rows,
+                                       int chunks_per_row, uint4 *xg) {
+    const int64_t total = (int64_t)n_rows * chunks_per_row;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / chunks_per_row, c = i - r * chunks_per_row;
+        xg[i] = x[(int64_t)row_tok[r] * chunks_per_row + c];
+    }
+}
 }  // namespace gq4

@@ -7,15 +7,19 @@
 // element), fp32 accumulation.
 //
 // Design (B200, HBM-bound):
-//  * Weights stay in the pages' layout, [O][I/2] bytes, low nibble first.  A warp takes
+//  * Weights: [O][I/2] bytes per matrix (rows as on the pages), nibbles of each 32-bit
+//    word in the device order described below.  A warp takes
 //    a 16-row x 64-column group tile (512 B): lane (g,t) reads 8 contiguous bytes of row
 //    g and of row g+8 -- every 32-byte sector is used whole.
 //  * The dot products run on the warp tensor op m16n8k16 (bf16 in, f32 out): the
-//    nibbles become exact bf16 integers (one lop3 + one bf16x2 fma per two weights), the
-//    16 contraction slots of one op are filled in an order chosen so that a lane's own
-//    bytes are its A fragment (no shuffles); the activations are staged once in shared
-//    memory in the matching order.  The op is only the dot-product engine: the bound
-//    is HBM, and this keeps the issue slots per weight near 1.
+//    nibbles become exact bf16 integers (one lop3 + one bf16x2 fma per two weights).
+//    The device word order (even-k nibbles in the low half-word, odd-k in the high one,
+//    written by gq4_upload) makes nibble slots i and i+4 of a word the bf16 pair of
+//    columns (2i, 2i+1); the 16 contraction slots of one op are assigned so that a
+//    lane's own 8 bytes are its A fragment (no shuffles) and its B fragment is 32
+//    contiguous bytes of the activation row, staged once in shared memory.  The op is
+//    only the dot-product engine: the bound is HBM, and this keeps the issue slots per
+//    weight near 1.
 //  * The f32 partial of each group is scaled by s[o][g] and added to the running sum.
 //  * A CTA (8 warps) owns a 16-row tile (32 with gate+up) for all columns it serves;
 //    its warps split the groups, and the eight partial tiles are summed in shared memory
@@ -63,21 +67,6 @@ struct ModeTraits {
 // Bytes of one staged column: the I activations as bf16 plus 16 B of padding, which
 // shifts consecutive columns by four banks (conflict-free 16-byte fragment reads).
 __host__ __device__ inline int skinny_xstride(int I) { return I * 2 + 16; }
-
-// Fragment order of 16 consecutive activations v[0..15] (eight bf16x2 words w[0..7],
-// w[i] = (v[2i], v[2i+1])): step j of the group uses (v0,v4),(v1,v5) / (v2,v6),(v3,v7) /
-// (v8,v12),(v9,v13) / (v10,v14),(v11,v15) -- the same pairing the nibble decode yields
-// for the weights (nibble i and nibble i+4 of a 32-bit word land in one bf16x2).
-__device__ __forceinline__ void frag_order16(const uint32_t (&w)[8], uint4 &o0, uint4 &o1) {
-    o0.x = __byte_perm(w[0], w[2], 0x5410);
-    o0.y = __byte_perm(w[0], w[2], 0x7632);
-    o0.z = __byte_perm(w[1], w[3], 0x5410);
-    o0.w = __byte_perm(w[1], w[3], 0x7632);
-    o1.x = __byte_perm(w[4], w[6], 0x5410);
-    o1.y = __byte_perm(w[4], w[6], 0x7632);
-    o1.z = __byte_perm(w[5], w[7], 0x5410);
-    o1.w = __byte_perm(w[5], w[7], 0x7632);
-}
 
 // Stage columns [c0, c0+nc) (nc <= xcols) of the activations into shared memory.
 template <int MODE>
@@ -127,11 +116,9 @@ __device__ __forceinline__ void skinny_stage(const SkinnyParams &p, char *xs, in
                 w[q * 2 + 1] = hb[2] | (hb[3] << 16);
             }
         }
-        uint4 o0, o1;
-        frag_order16(w, o0, o1);
         uint4 *dst = (uint4 *)(xs + (int64_t)cl * xstride + piece * 32);
-        dst[0] = o0;
-        dst[1] = o1;
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
 }
 
@@ -236,6 +223,7 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
                         }
                         #pragma unroll
                         for (int n = 0; n < NT; ++n) {
+                            if (n * 8 >= ncc) break;  // warp-uniform: no op for empty n-tiles
                             const int cl = cc + n * 8 + g;  // staged column this lane feeds
                             uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
                             if (n * 8 + g < ncc) {
