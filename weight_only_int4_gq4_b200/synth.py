@@ -130,7 +130,11 @@ MOE_PREFILL = MoEConfig("moe_prefill_t4096_h6144_e256_f2048_k8", T=4096, H=6144,
 MOE_BATCHED_E32 = MoEConfig("moe_batched_decode_t32_h6144_e32_f2048_k8", T=32, H=6144, E=32, F=2048,
                             K=8, seed=1003, sigma=float(np.sqrt(2.0)), n_hot=4, hot_bias=3.0)
 
-MOE_CONFIGS = {c.name: c for c in (MOE_DECODE, MOE_BATCHED, MOE_PREFILL, MOE_BATCHED_E32)}
+# profiling case of the prefill kernels: 128 rows per expert as at full size, 32 experts
+MOE_PREFILL_E32 = MoEConfig("moe_prefill_t512_h6144_e32_f2048_k8", T=512, H=6144, E=32, F=2048, K=8,
+                            seed=1004, oracle_sample=64)
+
+MOE_CONFIGS = {c.name: c for c in (MOE_DECODE, MOE_BATCHED, MOE_PREFILL, MOE_BATCHED_E32, MOE_PREFILL_E32)}
 
 DENSE_SHAPES = [(4096, 4096), (14336, 4096), (4096, 14336), (151936, 4096)]
 
