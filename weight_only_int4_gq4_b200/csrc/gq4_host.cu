@@ -262,14 +262,24 @@ bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Activation maps with 16/32/64/128-row boxes over a row-major bf16 [rows][cols] array.
+bool make_act_maps(CUtensorMap (&m)[4], const void *base, uint64_t cols, uint64_t rows) {
+    const uint32_t box_rows[4] = {16, 32, 64, 128};
+    for (int i = 0; i < 4; ++i)
+        if (!make_tmap_2d(&m[i], base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cols, rows, 64, box_rows[i],
+                          CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+    return true;
+}
+
 template <int MODE>
-gq4_status launch_tc(const CUtensorMap &w0, const CUtensorMap &w1, const CUtensorMap &x,
+gq4_status launch_tc(const CUtensorMap &w0, const CUtensorMap &w1, const CUtensorMap (&x)[4],
                      const TcParams &p, int units_upper, cudaStream_t st) {
     auto kern = gq4_tc_kernel<MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes) != cudaSuccess)
         return GQ4_ERR_CUDA;
     const int grid = std::max(1, std::min(units_upper, sm_count()));
-    kern<<<grid, kTcThreads, kTcSmemBytes, st>>>(w0, w1, x, p);
+    kern<<<grid, kTcThreads, kTcSmemBytes, st>>>(w0, w1, x[0], x[1], x[2], x[3], p);
     return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
 }
 
@@ -588,7 +598,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     if (st != GQ4_OK) return st;
 
     // experts with many rows: gathered activations, tensor-core gate+up and down
-    CUtensorMap tm_g, tm_u, tm_d, tm_x, tm_h;
+    CUtensorMap tm_g, tm_u, tm_d, tm_x[4], tm_h[4];
     TcParams tp{};
     if (tc) {
         const int max_large = std::max(1, std::min<int>(E, (int)(T * K / kLargeMin)));
@@ -598,11 +608,11 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
         if (cudaGetLastError() != cudaSuccess) return GQ4_ERR_CUDA;
         const uint64_t rows_gu = (uint64_t)(Wg->n_experts - 1) * (Wg->expert_stride_w / (H / 2)) + F;
         const uint64_t rows_d = (uint64_t)(Wd->n_experts - 1) * (Wd->expert_stride_w / (F / 2)) + H;
-        if (!make_tmap_2d(&tm_g, Wg->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H / 2, rows_gu, 32, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !make_tmap_2d(&tm_u, Wu->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H / 2, rows_gu, 32, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !make_tmap_2d(&tm_d, Wd->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, F / 2, rows_d, 32, 64, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !make_tmap_2d(&tm_x, at<void>(ws, L.xg), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, n, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tmap_2d(&tm_h, at<void>(ws, L.h), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, F, n, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+        // packed weights: 64-row boxes of 128 B (four groups), 128B-swizzled
+        if (!make_tmap_2d(&tm_g, Wg->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H / 2, rows_gu, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_2d(&tm_u, Wu->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H / 2, rows_gu, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_2d(&tm_d, Wd->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, F / 2, rows_d, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_act_maps(tm_x, at<void>(ws, L.xg), H, n) || !make_act_maps(tm_h, at<void>(ws, L.h), F, n))
             return GQ4_ERR_CUDA;
         tp.offs = at<int32_t>(ws, L.offs);
         tp.cnt = at<int32_t>(ws, L.cnt);

@@ -14,12 +14,18 @@
 //     the buffer -- the MMA of group g+1 overlaps the promotion of group g.
 // TMEM lane = weight row, so the scale is one register per thread and group.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over units):
-//   warp 0      TMA producer: packed nibble tile (128 rows x 32 B) and the activation
-//               tile (N <= 192 rows x 64 bf16, swizzle 128B) of each group into a 4-stage ring
-//   warp 1      TMEM allocation and the MMA issuer (one thread)
-//   warps 2-9   math: dequantise rows [16m, 16m+16) of the A tile, promote the TMEM
-//               partials of their lane quarter / column half, epilogue
+// Warp roles (512 threads = 4 warpgroups, one CTA per SM, persistent over units):
+//   WG0  warp 0  TMA producer of the packed nibble tiles: 128 rows x 128 B (four groups,
+//                swizzle 128B) per stage in two 64-row boxes, 5-stage ring
+//        warp 1  TMEM allocation and the MMA issuer (one thread)
+//        warp 2  TMA producer of the activation tiles (N <= 192 rows x 64 bf16, swizzle
+//                128B) as 128/64/32/16-row boxes, 4-stage ring; warp 3 idle
+//   (TMA cost is per request more than per byte: few large boxes keep the rings fed)
+//   WG1  warps 4-7   dequant: rows [32d, 32d+32) of the bf16 A tile, 4-slot ring
+//   WG2-3 warps 8-15 promotion: TMEM lane quarter (warp % 4) x column half, running
+//                sums in registers, epilogue
+// setmaxnreg moves registers from WG0/WG1 (48 each) to the promotion warps (200 each):
+// 256*48 + 256*200 = 63488 <= 65536 = 512 threads x 128 at launch.
 // Units: (large expert, M tile).  gate+up: an M tile is 64 gate rows + the same 64 up
 // rows, interleaved (A row 2i = gate row i, 2i+1 = up row i), so g and u of one output
 // sit in adjacent TMEM lanes of one warp and SiLU(g)*u needs one shuffle; down: 128 rows
@@ -33,18 +39,23 @@
 
 namespace gq4 {
 
-constexpr int kTcThreads = 320;
-constexpr int kTcStages = 4;
-constexpr int kTcAStages = 3;
+constexpr int kTcThreads = 512;
+constexpr int kTcWStages = 5;                                   // packed-weight ring, 4 groups/stage
+constexpr int kTcXStages = 4;                                   // activation ring, 1 group/stage
+constexpr int kTcAStages = 3;                                   // dequantised bf16 A tiles
 constexpr int kTcMaxN = 192;                                   // rows per pass (TMEM, registers)
 constexpr int kTcChunks = kTcMaxN / 64;                         // 32-column chunks per column half
-constexpr int kTcPackedBytes = 128 * 32;                        // 128 rows x 64 nibbles
+static_assert(kTcChunks == 3, "the promotion reads chunks 2c + half, c < 3");
+constexpr int kTcWGroups = 4;                                   // groups per weight stage
+constexpr int kTcWBytes = 128 * 32 * kTcWGroups;                // 128 rows x 256 nibbles
 constexpr int kTcXBytes = kTcMaxN * 128;                        // N rows x 64 bf16
-constexpr int kTcStageBytes = kTcPackedBytes + kTcXBytes;       // 36 KB, 1024-aligned
 constexpr int kTcABytes = 128 * 128;                            // 128 rows x 64 bf16
-constexpr int kTcOffA = kTcStages * kTcStageBytes;
-constexpr int kTcOffBar = kTcOffA + kTcAStages * kTcABytes;
-constexpr int kTcSmemBytes = kTcOffBar + 256 + 1024;            // + 1024 for alignment
+constexpr int kTcOffX = 0;                                      // 1024-aligned tiles first
+constexpr int kTcOffA = kTcOffX + kTcXStages * kTcXBytes;
+constexpr int kTcOffW = kTcOffA + kTcAStages * kTcABytes;
+constexpr int kTcOffBar = kTcOffW + kTcWStages * kTcWBytes;
+constexpr int kTcSmemBytes = kTcOffBar + 512 + 1024;            // + 1024 for alignment
+static_assert(kTcSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kTcTmemCols = 512;                                // two N<=192 partials (power of 2)
 constexpr int kStatusTimeout = 8;                               // GQ4_ERR_TIMEOUT
 
@@ -83,6 +94,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
+// As above, but the warp may be suspended in hardware (up to ~0.1 ms) until the phase
+// completes, instead of spinning on the issue slots the working warps need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(100000u) : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -94,8 +115,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63) == 0) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if ((i & 7) == 0) {
             if (*abort_flag) return false;
             if (global_ns() - t0 > 2000000000ull) {
                 *abort_flag = 1;
@@ -153,6 +174,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+// (a0, a1) += s * (p0, p1) as one packed f32x2 FMA.
+__device__ __forceinline__ void fma2(float &a0, float &a1, float p0, float p1, uint64_t ss) {
+    asm("{\n .reg .b64 ra, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rc, {%0, %1};\n"
+        " fma.rn.f32x2 rd, ra, %4, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+        : "+f"(a0), "+f"(a1) : "f"(p0), "f"(p1), "l"(ss));
+}
+__device__ __forceinline__ uint64_t splat2(float s) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(s));
+    return r;
+}
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -161,28 +193,36 @@ __device__ __forceinline__ void tmem_wait_ld() {
 template <int MODE>  // 0: gate+up with SiLU(g)*u -> h (bf16); 1: down -> y += w * D
 __global__ void __launch_bounds__(kTcThreads, 1)
 gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
-              const __grid_constant__ CUtensorMap tm_x, const TcParams p) {
+              const __grid_constant__ CUtensorMap tm_x16, const __grid_constant__ CUtensorMap tm_x32,
+              const __grid_constant__ CUtensorMap tm_x64, const __grid_constant__ CUtensorMap tm_x128,
+              const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
     const uint32_t bar0 = sb + kTcOffBar;
-    auto full_bar = [&](int s) { return bar0 + 8 * s; };
-    auto empty_bar = [&](int s) { return bar0 + 32 + 8 * s; };
-    auto afull_bar = [&](int a) { return bar0 + 64 + 8 * a; };
-    auto aempty_bar = [&](int a) { return bar0 + 88 + 8 * a; };
-    auto pfull_bar = [&](int b) { return bar0 + 112 + 8 * b; };
-    auto pempty_bar = [&](int b) { return bar0 + 128 + 8 * b; };
-    uint32_t *tmem_slot = (uint32_t *)(smem + kTcOffBar + 160);
-    volatile int *abort_flag = (volatile int *)(smem + kTcOffBar + 168);
+    auto wfull_bar = [&](int s) { return bar0 + 8 * s; };
+    auto wempty_bar = [&](int s) { return bar0 + 96 + 8 * s; };
+    auto xfull_bar = [&](int s) { return bar0 + 192 + 8 * s; };
+    auto xempty_bar = [&](int s) { return bar0 + 232 + 8 * s; };
+    auto afull_bar = [&](int a) { return bar0 + 272 + 8 * a; };
+    auto aempty_bar = [&](int a) { return bar0 + 296 + 8 * a; };
+    auto pfull_bar = [&](int b) { return bar0 + 320 + 8 * b; };
+    auto pempty_bar = [&](int b) { return bar0 + 336 + 8 * b; };
+    uint32_t *tmem_slot = (uint32_t *)(smem + kTcOffBar + 360);
+    volatile int *abort_flag = (volatile int *)(smem + kTcOffBar + 368);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTcStages; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1 + 8);
+        for (int s = 0; s < kTcWStages; ++s) {
+            mbar_init(wfull_bar(s), 1);
+            mbar_init(wempty_bar(s), 4);  // the four dequant warps
+        }
+        for (int s = 0; s < kTcXStages; ++s) {
+            mbar_init(xfull_bar(s), 1);
+            mbar_init(xempty_bar(s), 1);  // MMA commit
         }
         for (int a = 0; a < kTcAStages; ++a) {
-            mbar_init(afull_bar(a), 8);
+            mbar_init(afull_bar(a), 4);
             mbar_init(aempty_bar(a), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -204,9 +244,14 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
     const uint32_t tmem = *tmem_slot;
     const int n_units = (*p.n_large) * p.m_tiles;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+    if (warp < 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 48;" ::: "memory");
+      if (warp == 0 || warp == 2) {
+        // ------------------------------------------------------------ TMA producers
+        // warp 0: packed weights into the W ring; warp 2: activations into the X ring
         if (lane == 0) {
+            const bool wprod = warp == 0;
+            const int nst = wprod ? kTcWStages : kTcXStages;
             uint32_t it = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
@@ -216,36 +261,44 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                 const int wrow = e * p.estride_rows + (MODE == 0 ? mt * 64 : mt * 128);
                 for (int n0 = 0; ok && n0 < cnt; n0 += kTcMaxN) {
                     const int N = (min(kTcMaxN, cnt - n0) + 15) & ~15;
-                    for (int G = 0; G < p.ng; ++G, ++it) {
-                        const int s = it % kTcStages;
-                        if (!(ok = mbar_wait(empty_bar(s), ((it / kTcStages) & 1) ^ 1, abort_flag, p.status)))
-                            break;
-                        const uint32_t dst = sb + s * kTcStageBytes;
-                        mbar_expect_tx(full_bar(s), kTcPackedBytes + N * 128);
-                        if (MODE == 0) {
-                            tma_load_2d(dst, &tm_w0, G * 32, wrow, full_bar(s));
-                            tma_load_2d(dst + 2048, &tm_w1, G * 32, wrow, full_bar(s));
-                        } else {
-                            tma_load_2d(dst, &tm_w0, G * 32, wrow, full_bar(s));
-                            tma_load_2d(dst + 2048, &tm_w0, G * 32, wrow + 64, full_bar(s));
+                    if (wprod) {
+                        for (int G = 0; G < p.ng; G += kTcWGroups, ++it) {
+                            const int s = it % nst;
+                            if (!(ok = mbar_wait(wempty_bar(s), ((it / nst) & 1) ^ 1, abort_flag, p.status))) break;
+                            const uint32_t dst = sb + kTcOffW + s * kTcWBytes;
+                            mbar_expect_tx(wfull_bar(s), kTcWBytes);
+                            tma_load_2d(dst, &tm_w0, G * 32, wrow, wfull_bar(s));
+                            if (MODE == 0)
+                                tma_load_2d(dst + kTcWBytes / 2, &tm_w1, G * 32, wrow, wfull_bar(s));
+                            else
+                                tma_load_2d(dst + kTcWBytes / 2, &tm_w0, G * 32, wrow + 64, wfull_bar(s));
                         }
-                        for (int r = 0; r < N; r += 16)
-                            tma_load_2d(dst + kTcPackedBytes + r * 128, &tm_x, G * 64, row0 + n0 + r,
-                                        full_bar(s));
+                    } else {
+                        for (int G = 0; G < p.ng; ++G, ++it) {
+                            const int s = it % nst;
+                            if (!(ok = mbar_wait(xempty_bar(s), ((it / nst) & 1) ^ 1, abort_flag, p.status))) break;
+                            const uint32_t dst = sb + kTcOffX + s * kTcXBytes;
+                            mbar_expect_tx(xfull_bar(s), N * 128);
+                            int r = 0;  // N (a multiple of 16) as 128/64/32/16-row boxes
+                            if (N - r >= 128) { tma_load_2d(dst + r * 128, &tm_x128, G * 64, row0 + n0 + r, xfull_bar(s)); r += 128; }
+                            if (N - r >= 64) { tma_load_2d(dst + r * 128, &tm_x64, G * 64, row0 + n0 + r, xfull_bar(s)); r += 64; }
+                            if (N - r >= 32) { tma_load_2d(dst + r * 128, &tm_x32, G * 64, row0 + n0 + r, xfull_bar(s)); r += 32; }
+                            if (N - r >= 16) { tma_load_2d(dst + r * 128, &tm_x16, G * 64, row0 + n0 + r, xfull_bar(s)); r += 16; }
+                        }
                     }
                 }
             }
             if (!ok) {  // let copies already issued land before the CTA leaves
-                for (uint32_t j = it > kTcStages ? it - kTcStages : 0; j < it; ++j) {
+                for (uint32_t j = it > (uint32_t)nst ? it - nst : 0; j < it; ++j) {
+                    const uint32_t bar = wprod ? wfull_bar(j % nst) : xfull_bar(j % nst);
                     const uint64_t t0 = global_ns();
-                    while (!mbar_try_wait(full_bar(j % kTcStages), (j / kTcStages) & 1) &&
-                           global_ns() - t0 < 100000000ull) {
+                    while (!mbar_try_wait(bar, (j / nst) & 1) && global_ns() - t0 < 100000000ull) {
                     }
                 }
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             uint32_t it = 0;
@@ -258,97 +311,102 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                     const int N = (min(kTcMaxN, cnt - n0) + 15) & ~15;
                     const uint32_t idesc = idesc_bf16_m128(N);
                     for (int G = 0; G < p.ng; ++G, ++it) {
-                        const int s = it % kTcStages, as = it % kTcAStages, b = it & 1;
-                        ok = mbar_wait(full_bar(s), (it / kTcStages) & 1, abort_flag, p.status) &&
+                        const int xs = it % kTcXStages, as = it % kTcAStages, b = it & 1;
+                        ok = mbar_wait(xfull_bar(xs), (it / kTcXStages) & 1, abort_flag, p.status) &&
                              mbar_wait(afull_bar(as), (it / kTcAStages) & 1, abort_flag, p.status) &&
                              mbar_wait(pempty_bar(b), ((it >> 1) & 1) ^ 1, abort_flag, p.status);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t a_addr = sb + kTcOffA + as * kTcABytes;
-                        const uint32_t x_addr = sb + s * kTcStageBytes + kTcPackedBytes;
+                        const uint32_t x_addr = sb + kTcOffX + xs * kTcXBytes;
                         #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             tc_mma(tmem + b * 256, sw128_desc(a_addr + kk * 32),
                                    sw128_desc(x_addr + kk * 32), idesc, kk > 0 ? 1u : 0u);
                         tc_commit(pfull_bar(b));
                         tc_commit(aempty_bar(as));
-                        tc_commit(empty_bar(s));
+                        tc_commit(xempty_bar(xs));
                     }
                 }
             }
             // the last commits must have arrived before the CTA's shared memory is released
             if (ok && it > 0) {
                 const uint32_t j = it - 1;
-                mbar_wait(empty_bar(j % kTcStages), (j / kTcStages) & 1, abort_flag, p.status);
+                mbar_wait(xempty_bar(j % kTcXStages), (j / kTcXStages) & 1, abort_flag, p.status);
                 mbar_wait(aempty_bar(j % kTcAStages), (j / kTcAStages) & 1, abort_flag, p.status);
             }
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------ math warps
-        const int m = warp - 2;            // 0..7: A rows [16m, 16m+16)
-        const int q = warp & 3;            // TMEM lane quarter this warp may access
-        const int half = m >> 2;           // column half: 32-column chunks 2c + half
-        const int lrow = 32 * q + lane;    // TMEM lane = A row owned in the promotion
-        const int drow = 16 * m + (lane >> 1), dkh = lane & 1;  // dequant: A row, k half
+      } else if (warp >= 4) {
+        // ------------------------------------------------------------ dequant warps
+        // A row written by this lane.  Lanes l and rows pair up so that the eight lanes
+        // of a shared-memory phase hit eight distinct 16-byte swizzle slots both when
+        // reading the packed tile (slot = prow & 7) and when writing the A row (r & 7).
+        const int l16 = lane & 15;
+        const int r16 = l16 < 8 ? 2 * l16 + (l16 >> 2) : 2 * (l16 - 8) + 1 - ((l16 - 8) >> 2);
+        const int r = 32 * (warp - 4) + 16 * (lane >> 4) + r16;
         // packed tile rows: [0,64) first box, [64,128) second; gate+up interleaves them
-        const int prow = MODE == 0 ? ((drow & 1) ? 64 + (drow >> 1) : (drow >> 1)) : drow;
+        const int prow = MODE == 0 ? ((r & 1) ? 64 + (r >> 1) : (r >> 1)) : r;
+        uint32_t it = 0, wit = 0;  // group counter, weight-stage counter
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+            const int e = p.large[u / p.m_tiles];
+            const int cnt = p.cnt[e];
+            for (int n0 = 0; ok && n0 < cnt; n0 += kTcMaxN) {
+                for (int G = 0; G < p.ng; ++G, ++it) {
+                    const uint32_t wi = wit + (G >> 2);  // weight stage of this group
+                    const int ws = wi % kTcWStages, as = it % kTcAStages;
+                    if ((G & 3) == 0 &&
+                        !(ok = mbar_wait(wfull_bar(ws), (wi / kTcWStages) & 1, abort_flag, p.status)))
+                        break;
+                    if (!(ok = mbar_wait(aempty_bar(as), ((it / kTcAStages) & 1) ^ 1, abort_flag, p.status)))
+                        break;
+                    // packed tile (128B-swizzled): row pr at pr*128, its 16-byte chunk c at
+                    // (c ^ (pr & 7)) * 16; group G%4 is chunks 2(G%4), 2(G%4)+1; rows
+                    // [64,128) in the second half
+                    const uint8_t *wrow_p = smem + kTcOffW + ws * kTcWBytes + (prow >> 6) * (kTcWBytes / 2) +
+                                            (prow & 63) * 128;
+                    const int c0 = 2 * (G & 3), swz = prow & 7;
+                    const uint4 w0 = *(const uint4 *)(wrow_p + ((c0 ^ swz) << 4));
+                    const uint4 w1 = *(const uint4 *)(wrow_p + (((c0 + 1) ^ swz) << 4));
+                    if ((G & 3) == 3) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(wempty_bar(ws));  // all four groups read
+                    }
+                    uint8_t *arow = smem + kTcOffA + as * kTcABytes + r * 128;
+                    const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    #pragma unroll
+                    for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = columns 8c..8c+7
+                        uint4 o;
+                        o.x = nib2_to_bf16x2(wv[c]);
+                        o.y = nib2_to_bf16x2(wv[c] >> 4);
+                        o.z = nib2_to_bf16x2(wv[c] >> 8);
+                        o.w = nib2_to_bf16x2(wv[c] >> 12);
+                        *(uint4 *)(arow + ((c ^ (r & 7)) << 4)) = o;
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(afull_bar(as));
+                }
+                wit += p.ng / kTcWGroups;
+            }
+        }
+      }
+    } else {
+        // ------------------------------------------------------------ promotion warps
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+        const int q = warp & 3;              // TMEM lane quarter this warp may access
+        const int half = (warp - 8) >> 2;    // column half: 32-column chunks 2c + half
+        const int lrow = 32 * q + lane;      // TMEM lane = A row
         uint32_t it = 0;
         bool ok = true;
         float acc[kTcChunks][32];
-
-        auto dequant = [&](uint32_t i) -> bool {
-            const int s = i % kTcStages, as = i % kTcAStages;
-            if (!mbar_wait(full_bar(s), (i / kTcStages) & 1, abort_flag, p.status)) return false;
-            if (!mbar_wait(aempty_bar(as), ((i / kTcAStages) & 1) ^ 1, abort_flag, p.status)) return false;
-            const uint4 w = *(const uint4 *)(smem + s * kTcStageBytes + prow * 32 + dkh * 16);
-            uint8_t *arow = smem + kTcOffA + as * kTcABytes + drow * 128;
-            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-            #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int c = dkh * 4 + j;  // 16-byte chunk = columns 8c..8c+7
-                uint4 o;
-                o.x = nib2_to_bf16x2(wv[j]);
-                o.y = nib2_to_bf16x2(wv[j] >> 4);
-                o.z = nib2_to_bf16x2(wv[j] >> 8);
-                o.w = nib2_to_bf16x2(wv[j] >> 12);
-                *(uint4 *)(arow + ((c ^ (drow & 7)) << 4)) = o;
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(afull_bar(as));
-                mbar_arrive(empty_bar(s));
-            }
-            return true;
-        };
-        auto promote = [&](uint32_t i, float scale, int N) -> bool {
-            const int b = i & 1;
-            if (!mbar_wait(pfull_bar(b), (i >> 1) & 1, abort_flag, p.status)) return false;
-            tc_fence_after();
-            #pragma unroll
-            for (int c = 0; c < kTcChunks; ++c) {
-                const int col = 32 * (2 * c + half);
-                if (col < N) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + b * 256 + col, r);
-                    tmem_wait_ld();
-                    #pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[c][j] = fmaf(scale, __uint_as_float(r[j]), acc[c][j]);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(pempty_bar(b));
-            return true;
-        };
 
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
             const int a = u / p.m_tiles, mt = u - a * p.m_tiles;
             const int e = p.large[a];
             const int row0 = p.offs[e], cnt = p.cnt[e];
-            // the scale row of this thread's TMEM lane
-            const float *srow;
+            const float *srow;  // the scale row of this thread's TMEM lane
             if (MODE == 0)
                 srow = ((lrow & 1) ? p.s1 : p.s0) + (int64_t)e * p.estride_s +
                        (int64_t)(mt * 64 + (lrow >> 1)) * p.ng;
@@ -361,17 +419,59 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                 for (int c = 0; c < kTcChunks; ++c)
                     #pragma unroll
                     for (int j = 0; j < 32; ++j) acc[c][j] = 0.f;
-                float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                float prev_scale = 0.f;
-                for (int G = 0; G < p.ng; ++G) {
-                    if (!(ok = dequant(it + G))) break;
-                    if ((G & 3) == 0) s4 = *(const float4 *)(srow + G);  // ng % 4 == 0
-                    const float sc = (G & 3) == 0 ? s4.x : (G & 3) == 1 ? s4.y : (G & 3) == 2 ? s4.z : s4.w;
-                    if (G > 0 && !(ok = promote(it + G - 1, prev_scale, N))) break;
-                    prev_scale = sc;
+                // scales four groups at a time, prefetched one float4 ahead (ng % 4 == 0)
+                float4 s_cur = *(const float4 *)srow;
+                float4 s_next = p.ng > 4 ? *(const float4 *)(srow + 4) : s_cur;
+                for (int G = 0; G < p.ng; ++G, ++it) {
+                    const int gq = G & 3;
+                    const float sc = gq == 0 ? s_cur.x : gq == 1 ? s_cur.y : gq == 2 ? s_cur.z : s_cur.w;
+                    if (gq == 3) {
+                        s_cur = s_next;
+                        if (G + 5 < p.ng) s_next = *(const float4 *)(srow + G + 5);
+                    }
+                    const int b = it & 1;
+                    if (!(ok = mbar_wait(pfull_bar(b), (it >> 1) & 1, abort_flag, p.status))) break;
+                    tc_fence_after();
+                    const uint64_t ss = splat2(sc);
+                    const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + b * 256;
+                    // chunks 2c + half of 32 columns; the first two are loaded together
+                    const int col0 = 32 * half, col1 = 32 * (2 + half), col2 = 32 * (4 + half);
+                    if (col0 < N) {
+                        uint32_t r0[32], r1[32];
+                        tmem_ld32(tbase + col0, r0);
+                        if (col1 < N) tmem_ld32(tbase + col1, r1);
+                        tmem_wait_ld();
+                        if (col2 >= N) {  // nothing else to read: the buffer may be reused
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(pempty_bar(b));
+                        }
+                        #pragma unroll
+                        for (int j = 0; j < 32; j += 2)
+                            fma2(acc[0][j], acc[0][j + 1], __uint_as_float(r0[j]), __uint_as_float(r0[j + 1]), ss);
+                        if (col1 < N) {
+                            #pragma unroll
+                            for (int j = 0; j < 32; j += 2)
+                                fma2(acc[1][j], acc[1][j + 1], __uint_as_float(r1[j]), __uint_as_float(r1[j + 1]), ss);
+                        }
+                    }
+                    if (col2 < N) {
+                        uint32_t r2[32];
+                        tmem_ld32(tbase + col2, r2);
+                        tmem_wait_ld();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(pempty_bar(b));
+                        #pragma unroll
+                        for (int j = 0; j < 32; j += 2)
+                            fma2(acc[2][j], acc[2][j + 1], __uint_as_float(r2[j]), __uint_as_float(r2[j + 1]), ss);
+                    }
+                    if (half == 1 && N <= 32) {  // this warp owns no chunk of this pass
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(pempty_bar(b));
+                    }
                 }
-                if (ok) ok = promote(it + p.ng - 1, prev_scale, N);
-                it += p.ng;
                 if (!ok) break;
                 // ---------------------------------------------------- epilogue
                 if (MODE == 0) {
@@ -398,14 +498,19 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                     for (int c = 0; c < kTcChunks; ++c) {
                         const int col = 32 * (2 * c + half);
                         if (col < N) {
+                            // token and weight of the 32 columns: one coalesced load per lane
+                            int tok_l = 0;
+                            float wt_l = 0.f;
+                            if (col + lane < nrows) {
+                                const int rr = row0 + n0 + col + lane;
+                                tok_l = p.row_tok[rr];
+                                wt_l = p.wts[p.row_slot[rr]];
+                            }
                             #pragma unroll
                             for (int j = 0; j < 32; ++j) {
-                                if (col + j < nrows) {
-                                    const int r = row0 + n0 + col + j;
-                                    const int tok = p.row_tok[r];
-                                    const float wt = p.wts[p.row_slot[r]];
-                                    atomicAdd(p.y + (int64_t)tok * p.O + o, wt * acc[c][j]);
-                                }
+                                const int tok = __shfl_sync(0xffffffffu, tok_l, j);
+                                const float wt = __shfl_sync(0xffffffffu, wt_l, j);
+                                if (col + j < nrows) atomicAdd(p.y + (int64_t)tok * p.O + o, wt * acc[c][j]);
                             }
                         }
                     }
