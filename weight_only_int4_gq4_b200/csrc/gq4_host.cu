@@ -114,6 +114,35 @@ gq4_status launch_skinny(SkinnyParams p, int max_cols, bool f32x, int units_uppe
     }
 }
 
+// Row-band kernel for 3..32 (or more, in passes) bf16 activation columns.
+template <int MODE, int NT>
+gq4_status launch_band_nt(const SkinnyParams &p, int units_upper, int32_t *status, cudaStream_t st) {
+    auto kern = gq4_band_kernel<MODE, NT>;
+    const size_t smem = band_smem(ModeTraits<MODE>::kPair);
+    if (allow_smem(kern, smem) != cudaSuccess) return GQ4_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess)
+        return GQ4_ERR_CUDA;
+    per_sm = std::max(per_sm, 1);
+    const int grid = std::max(1, std::min(units_upper, per_sm * sm_count()));
+    kern<<<grid, 256, smem, st>>>(p, status);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
+template <int MODE>
+gq4_status launch_band(const SkinnyParams &p, int max_cols, int units_upper, int32_t *status,
+                       cudaStream_t st) {
+    const int c = std::min(max_cols, kBandMaxCols);
+    if (c <= 8) return launch_band_nt<MODE, 1>(p, units_upper, status, st);
+    if (c <= 16) return launch_band_nt<MODE, 2>(p, units_upper, status, st);
+    if (c <= 24) return launch_band_nt<MODE, 3>(p, units_upper, status, st);
+    return launch_band_nt<MODE, 4>(p, units_upper, status, st);
+}
+
+// Decode-path dispatch: the row-band kernel from 3 bf16 columns on, the split-K kernel
+// for one or two columns (where bands would leave most SMs idle) and for f32 columns.
+constexpr int kBandMinCols = 3;
+
 // ---- MoE workspace layout --------------------------------------------------------------
 struct MoeLayout {
     size_t status, idx, wts, cnt, offs, row_tok, row_slot, slot_row, n_active, active, chunk,
@@ -401,6 +430,8 @@ gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.y = y;
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    if (xdt == GQ4_BF16 && n_tok >= kBandMinCols)
+        return launch_band<kMatvec>(p, cols, (p.row_tiles + 7) / 8, nullptr, S(stream));
     return launch_skinny<kMatvec>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
 }
 
@@ -428,6 +459,8 @@ gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const vo
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.h = h;
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    if (xdt == GQ4_BF16 && n_tok >= kBandMinCols)
+        return launch_band<kGateUp>(p, cols, (p.row_tiles + 7) / 8, nullptr, S(stream));
     return launch_skinny<kGateUp>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
 }
 
@@ -594,7 +627,10 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     pg.zero_ptr = y; pg.zero_n = T * H;
     if ((T * H) % 4) return GQ4_ERR_SHAPE;
     const int small_cols = (int)std::min<int64_t>(max_cols, tc ? kLargeMin - 1 : max_cols);
-    st = launch_skinny<kMoeGateUp>(pg, small_cols, false, max_active * pg.row_tiles, s);
+    const bool band = small_cols >= kBandMinCols;
+    int32_t *status = at<int32_t>(ws, L.status);
+    st = band ? launch_band<kMoeGateUp>(pg, small_cols, max_active * ((pg.row_tiles + 7) / 8), status, s)
+              : launch_skinny<kMoeGateUp>(pg, small_cols, false, max_active * pg.row_tiles, s);
     if (st != GQ4_OK) return st;
 
     // experts with many rows: gathered activations, tensor-core gate+up and down
@@ -640,7 +676,8 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     pd.row_tiles = (int)((H + 15) / 16);
     pd.x = at<void>(ws, L.h); pd.xdt = 1; pd.n_tok = (int)T;
     pd.y = y;
-    st = launch_skinny<kMoeDown>(pd, small_cols, false, max_active * pd.row_tiles, s);
+    st = band ? launch_band<kMoeDown>(pd, small_cols, max_active * ((pd.row_tiles + 7) / 8), status, s)
+              : launch_skinny<kMoeDown>(pd, small_cols, false, max_active * pd.row_tiles, s);
     if (st != GQ4_OK) return st;
     if (tc) {
         const int max_large = std::max(1, std::min<int>(E, (int)(T * K / kLargeMin)));

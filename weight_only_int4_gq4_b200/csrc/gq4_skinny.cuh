@@ -315,3 +315,263 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
 }
 
 }  // namespace gq4
+
+// ======================================================================================
+// Row-band decode kernel (3 or more activation columns per matrix/expert).
+//
+// A CTA owns a band of 8 row tiles (one per warp; 128 rows, or 128 gate + 128 up rows)
+// of one matrix/expert for all of K, so the activations of the expert's rows are read
+// once per band instead of once per row tile, and no cross-warp reduction is needed:
+//  * activations: chunks of kBandKC groups (512 columns) of the expert's rows, one bulk
+//    copy per row (the copy's source does the token gather), double-buffered, completion
+//    on an mbarrier with a transaction count;
+//  * weights and scales: each warp streams its own 16-row tiles through a private
+//    kBandDW-stage shared-memory ring with cp.async (rows past O are zero-filled), kBandDW-1
+//    groups ahead of the tensor ops;
+//  * products: the same nibble decode and m16n8k16 fragments as the split-K kernel.
+// ======================================================================================
+namespace gq4 {
+
+constexpr int kBandKC = 8;      // groups per activation chunk
+constexpr int kBandDW = 8;      // per-warp weight ring depth (groups)
+constexpr int kBandMaxCols = 32;
+__host__ __device__ inline int band_xstride() { return kBandKC * 64 * 2 + 16; }  // bytes per staged row
+__host__ __device__ inline int band_wstage(int pair) { return pair * (16 * 32 + 16 * 4); }
+__host__ __device__ inline size_t band_smem(int pair) {
+    return (size_t)2 * kBandMaxCols * band_xstride() + (size_t)8 * kBandDW * band_wstage(pair) + 64;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+// Bounded wait (about two seconds of SM cycles); false if it gave up.
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t ok;
+        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+                     " selp.u32 %0, 1, 0, p;\n}\n" : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > 4000000000ll) return false;
+    }
+}
+
+template <int MODE, int NT>
+__global__ void __launch_bounds__(256) gq4_band_kernel(const SkinnyParams p, int32_t *status) {
+    using TR = ModeTraits<MODE>;
+    constexpr int PAIR = TR::kPair;
+    extern __shared__ __align__(128) uint8_t bsm[];
+    const int xstride = band_xstride();
+    uint8_t *xbuf = bsm;                                                   // [2][32 rows][xstride]
+    uint8_t *wring = bsm + 2 * kBandMaxCols * xstride;                     // [8 warps][DW][stage]
+    const uint32_t xbar = smem_addr(wring + 8 * kBandDW * band_wstage(PAIR)); // 2 mbarriers
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int rb = p.I >> 1;
+    const int wst = band_wstage(PAIR);
+    uint8_t *myring = wring + warp * kBandDW * wst;
+    const int bands = (p.row_tiles + 7) >> 3;
+    const int nchunks = (p.ng + kBandKC - 1) / kBandKC;
+
+    if (threadIdx.x == 0) {
+        bar_init(xbar, 1);
+        bar_init(xbar + 8, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (MODE == kMoeGateUp && p.zero_ptr) {
+        float4 *z = (float4 *)p.zero_ptr;
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_n / 4;
+             i += (int64_t)gridDim.x * blockDim.x)
+            z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+
+    const int n_units = TR::kMoe ? (*p.n_active) * bands : bands;
+    uint32_t xphase[2] = {0u, 0u};
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        int e = 0, band = u, row0 = 0, cols = p.n_tok;
+        if (TR::kMoe) {
+            const int a = u / bands;
+            band = u - a * bands;
+            e = p.active[a];
+            row0 = p.offs[e];
+            cols = p.cnt[e];
+        }
+        const int rt = band * 8 + warp;          // this warp's row tile
+        const bool tile_ok = rt < p.row_tiles;
+        const uint8_t *W0 = p.w0 + (int64_t)e * p.estride_w;
+        const float *S0 = p.s0 + (int64_t)e * p.estride_s;
+        const uint8_t *W1 = PAIR == 2 ? p.w1 + (int64_t)e * p.estride_w : nullptr;
+        const float *S1 = PAIR == 2 ? p.s1 + (int64_t)e * p.estride_s : nullptr;
+
+        for (int c0 = 0; c0 < cols; c0 += kBandMaxCols) {
+            const int nc = min(kBandMaxCols, cols - c0);
+            // weight prefetch of group G into ring slot G % DW (one commit group per group)
+            auto issue_w = [&](int G) {
+                if (G < p.ng && tile_ok) {
+                    uint8_t *st = myring + (G % kBandDW) * wst;
+                    #pragma unroll
+                    for (int m = 0; m < PAIR; ++m) {
+                        const uint8_t *Wm = m ? W1 : W0;
+                        const float *Sm = m ? S1 : S0;
+                        const int row = rt * 16 + (lane >> 1);
+                        const bool rv = row < p.O;
+                        const uint8_t *src = Wm + (int64_t)(rv ? row : 0) * rb + (int64_t)G * 32 + (lane & 1) * 16;
+                        cp_async16(smem_addr(st + m * 576 + (lane >> 1) * 32 + (lane & 1) * 16), src, rv ? 16u : 0u);
+                        if (lane < 16) {
+                            const int srow = rt * 16 + lane;
+                            const bool sv = srow < p.O;
+                            cp_async4(smem_addr(st + m * 576 + 512 + lane * 4), Sm + (int64_t)(sv ? srow : 0) * p.ng + G,
+                                      sv ? 4u : 0u);
+                        }
+                    }
+                }
+                cp_async_commit();  // possibly empty: keeps the group count uniform
+            };
+            // activation chunk c of rows [c0, c0+nc) into buffer c & 1
+            auto issue_x = [&](int c) {
+                if (c < nchunks && warp == 0) {
+                    const int k0 = c * kBandKC * 64;
+                    const int kn = min(kBandKC * 64, p.I - k0);
+                    const uint32_t bar = xbar + 8 * (c & 1);
+                    if (lane == 0) bar_expect_tx(bar, (uint32_t)(nc * kn * 2));
+                    __syncwarp();
+                    for (int r = lane; r < nc; r += 32) {
+                        const int col = c0 + r;
+                        const uint16_t *src;
+                        if (MODE == kMoeGateUp)
+                            src = (const uint16_t *)p.x + (int64_t)p.row_tok[row0 + col] * p.I + k0;
+                        else if (MODE == kMoeDown)
+                            src = (const uint16_t *)p.x + (int64_t)(row0 + col) * p.I + k0;
+                        else
+                            src = (const uint16_t *)p.x + (int64_t)col * p.I + k0;
+                        bulk_g2s(smem_addr(xbuf + ((c & 1) * kBandMaxCols + r) * xstride), src, kn * 2, bar);
+                    }
+                }
+            };
+
+            float acc[PAIR][NT][4];
+            #pragma unroll
+            for (int m = 0; m < PAIR; ++m)
+                #pragma unroll
+                for (int n = 0; n < NT; ++n)
+                    #pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+
+            issue_x(0);
+            #pragma unroll
+            for (int G = 0; G < kBandDW - 1; ++G) issue_w(G);
+            for (int c = 0; c < nchunks; ++c) {
+                issue_x(c + 1);
+                const uint32_t bar = xbar + 8 * (c & 1);
+                const bool late = !bar_wait(bar, xphase[c & 1]);
+                xphase[c & 1] ^= 1u;
+                const uint8_t *xc = xbuf + (c & 1) * kBandMaxCols * xstride;
+                const int gend = min(p.ng, (c + 1) * kBandKC);
+                for (int G = c * kBandKC; G < gend; ++G) {
+                    __syncwarp();                  // slot (G-1) % DW is read by every lane
+                    issue_w(G + kBandDW - 1);
+                    cp_async_wait<kBandDW - 1>();  // group G has landed (this thread's copies)
+                    __syncwarp();                  // ... and every lane's
+                    if (!tile_ok) continue;
+                    const uint8_t *st = myring + (G % kBandDW) * wst;
+                    const int gl = G - c * kBandKC;
+                    uint32_t ra[PAIR][8], rbv[PAIR][8];
+                    float sa[PAIR], sb[PAIR];
+                    #pragma unroll
+                    for (int m = 0; m < PAIR; ++m) {
+                        const uint2 wa = *(const uint2 *)(st + m * 576 + g * 32 + t * 8);
+                        const uint2 wb = *(const uint2 *)(st + m * 576 + (g + 8) * 32 + t * 8);
+                        sa[m] = *(const float *)(st + m * 576 + 512 + g * 4);
+                        sb[m] = *(const float *)(st + m * 576 + 512 + (g + 8) * 4);
+                        #pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            ra[m][i] = nib2_to_bf16x2(wa.x >> (4 * i));
+                            ra[m][4 + i] = nib2_to_bf16x2(wa.y >> (4 * i));
+                            rbv[m][i] = nib2_to_bf16x2(wb.x >> (4 * i));
+                            rbv[m][4 + i] = nib2_to_bf16x2(wb.y >> (4 * i));
+                        }
+                    }
+                    #pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        if (n * 8 >= nc) break;  // warp-uniform
+                        uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+                        if (n * 8 + g < nc) {
+                            const uint4 *src = (const uint4 *)(xc + (n * 8 + g) * xstride + (gl * 4 + t) * 32);
+                            b0 = src[0];
+                            b1 = src[1];
+                        }
+                        const uint32_t bf[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                        #pragma unroll
+                        for (int m = 0; m < PAIR; ++m) {
+                            float d[4] = {0.f, 0.f, 0.f, 0.f};
+                            #pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint32_t a[4] = {ra[m][2 * j], rbv[m][2 * j], ra[m][2 * j + 1], rbv[m][2 * j + 1]};
+                                mma_bf16_16816(d, a, bf[2 * j], bf[2 * j + 1], d);
+                            }
+                            acc[m][n][0] = fmaf(sa[m], d[0], acc[m][n][0]);
+                            acc[m][n][1] = fmaf(sa[m], d[1], acc[m][n][1]);
+                            acc[m][n][2] = fmaf(sb[m], d[2], acc[m][n][2]);
+                            acc[m][n][3] = fmaf(sb[m], d[3], acc[m][n][3]);
+                        }
+                    }
+                }
+                // every warp is done with buffer c & 1; a wait that gave up anywhere ends
+                // the CTA (GQ4_ERR_TIMEOUT) once the copies it issued have landed or timed out
+                if (__syncthreads_or(late)) {
+                    if (threadIdx.x == 0 && status) atomicOr(status, 8);
+                    bar_wait(bar, xphase[c & 1] ^ 1u);
+                    if (c + 1 < nchunks) bar_wait(xbar + 8 * ((c + 1) & 1), xphase[(c + 1) & 1]);
+                    cp_async_wait<0>();
+                    return;
+                }
+            }
+            cp_async_wait<0>();
+            // ---------------------------------------------------------------- epilogue
+            if (tile_ok) {
+                #pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    #pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int cl = n * 8 + 2 * t + (i & 1);
+                        const int o = rt * 16 + g + ((i >> 1) << 3);
+                        if (cl >= nc || o >= p.O) continue;
+                        const int c = c0 + cl;
+                        if (MODE == kMatvec) {
+                            p.y[(int64_t)c * p.O + o] = acc[0][n][i];
+                        } else if (MODE == kGateUp) {
+                            ((uint16_t *)p.h)[(int64_t)c * p.O + o] =
+                                (uint16_t)bf16_bits_rn(silu_mul(acc[0][n][i], acc[PAIR - 1][n][i]));
+                        } else if (MODE == kMoeGateUp) {
+                            ((uint16_t *)p.h)[(int64_t)(row0 + c) * p.O + o] =
+                                (uint16_t)bf16_bits_rn(silu_mul(acc[0][n][i], acc[PAIR - 1][n][i]));
+                        } else {
+                            const int r = row0 + c;
+                            atomicAdd(p.y + (int64_t)p.row_tok[r] * p.O + o, p.wts[p.row_slot[r]] * acc[0][n][i]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+}
+
+}  // namespace gq4
