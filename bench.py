@@ -141,18 +141,63 @@ def cpu_baseline(cfg: synth.MoEConfig, budget_s: float = 12.0, max_tokens: int =
                       f"{elapsed:.1f} s, fp64 plain C"}
 
 
-def alg_bytes(cfg, n_active):
-    """Algorithmic HBM bytes per step: packed weights + scales of the experts touched,
-    plus activations, logits, h and y traffic."""
-    per_w = lambda O, I: O * (I // 2) + O * (I // 64) * 4  # noqa: E731
-    gate_up = n_active * 2 * per_w(cfg.F, cfg.H)
-    down = n_active * per_w(cfg.H, cfg.F)
+def per_matrix_bytes(O, I):
+    """Packed nibbles plus f32 group scales of one [O][I] matrix."""
+    return O * (I // 2) + O * (I // 64) * 4
+
+
+def split_experts(cfg, cnt):
+    """The experts moe_expert_ffn sends to the tensor-core kernels (at least
+    GQ4_MOE_LARGE_MIN_ROWS rows, when T and the shapes allow) and to the decode kernels."""
+    from weight_only_int4_gq4_b200 import gq4
+    lim = gq4.MOE_LARGE_MIN_ROWS
+    tc = cfg.T >= lim and cfg.H % 128 == 0 and cfg.F % 64 == 0
+    large = (cnt >= lim) if tc else np.zeros(cnt.shape, bool)
+    small = (cnt > 0) & ~large
+    return {"tc": tc, "n_small": int(small.sum()), "rows_small": int(cnt[small].sum()),
+            "n_large": int(large.sum()), "rows_large": int(cnt[large].sum())}
+
+
+STAGES = ("route_rowmap", "gate_up_small", "gate_up_large", "down_small", "down_large")
+
+
+def stage_work(cfg, sp):
+    """Algorithmic HBM bytes and tensor-core FLOPs of each timed stage of one step:
+    weights + scales of the experts the stage serves, the activations it must read once,
+    the outputs it must write.  The row gather before the tensor-core gate+up is an
+    implementation choice: its time is in the stage, its bytes are not."""
+    H, F, T, n = cfg.H, cfg.F, cfg.T, cfg.T * cfg.K
+    rs, rl = sp["rows_small"], sp["rows_large"]
+    y_rmw = 2 * T * H * 4
+    fs = rs / max(rs + rl, 1)
+    w = {
+        "route_rowmap": (T * cfg.E * 4 + n * 20 + cfg.E * 8, 0.0),
+        "gate_up_small": (sp["n_small"] * 2 * per_matrix_bytes(F, H) + (T * H * 2 if rs else 0)
+                          + rs * F * 2 + T * H * 4, 0.0),
+        "gate_up_large": (sp["n_large"] * 2 * per_matrix_bytes(F, H) + (T * H * 2 if rl else 0)
+                          + rl * F * 2, 2.0 * rl * 2 * F * H),
+        "down_small": (sp["n_small"] * per_matrix_bytes(H, F) + rs * F * 2 + fs * y_rmw, 0.0),
+        "down_large": (sp["n_large"] * per_matrix_bytes(H, F) + rl * F * 2 + (1 - fs) * y_rmw,
+                       2.0 * rl * H * F),
+    }
+    return w
+
+
+def stage_kernels(cfg, sp):
+    few = "gq4_band_kernel" if min(cfg.T, 23 if sp["tc"] else cfg.T) >= 3 else "gq4_skinny_kernel"
     n = cfg.T * cfg.K
-    x = cfg.T * cfg.H * 2
-    h = n * cfg.F * 2
-    y = cfg.T * cfg.H * 4
-    return {"gate_up": gate_up + x + h, "down": down + h + y * 2, "step": gate_up + down + x + 2 * h + 2 * y
-            + cfg.T * cfg.E * 4}
+    route = "gq4_route_rowmap_small_kernel" if n <= 1024 else \
+        "gq4_route_kernel + gq4_rowmap_{count,scan,fill}_kernel"
+    return {"route_rowmap": route, "gate_up_small": f"{few}<MoeGateUp>",
+            "gate_up_large": "gq4_gather_rows_kernel + gq4_tc_kernel<GateUp>",
+            "down_small": f"{few}<MoeDown>", "down_large": "gq4_tc_kernel<Down>"}
+
+
+def launches_per_step(cfg, sp):
+    """Kernels of this library one moe_expert_ffn call launches (the status memset is a
+    runtime memset, not counted)."""
+    n = cfg.T * cfg.K
+    return (1 if n <= 1024 else 4) + 2 + (3 if sp["tc"] else 0)
 
 
 def run_reference(args, cfg, rank):
@@ -222,7 +267,7 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     n_slots = cfg.T * cfg.K
-    launches_per_step = 3 if n_slots <= 1024 else 6
+    NEV = gq4.MOE_STAGE_EVENTS
 
     def step(ev=None):
         gq4.moe_expert_ffn(Wg, Wu, Wd, logits, x, cfg.K, y=y, ws=ws, stage_events=ev)
@@ -230,11 +275,12 @@ def main():
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    n_active = int(ws.routing()["n_active"].cpu()[0])
     assert ws.status() == 0
+    cnt = ws.routing()["cnt"].cpu().numpy()[:cfg.E]
+    split = split_experts(cfg, cnt)
 
     # ---- device-timed steps (L2 flushed between steps, outside the events)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NEV)] for _ in range(args.steps)]
     for row in evs:  # torch creates the CUDA event lazily, at its first record
         for e in row:
             e.record(stream)
@@ -248,7 +294,8 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)])
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(NEV - 1)]
+                      for i in range(args.steps)])
     step_ms = stage.sum(1)
     ms = float(step_ms.mean())
 
@@ -279,18 +326,31 @@ def main():
     ms, e2e = float(t[0]), float(t[1])
 
     hbm, bf16, peak_kind = peaks()
-    ab = alg_bytes(cfg, n_active)
-    t_gu = float(stage[:, 1].mean())
-    t_dn = float(stage[:, 2].mean())
-    dominant = ("gate_up", t_gu) if t_gu >= t_dn else ("down", t_dn)
-    achieved = ab[dominant[0]] / (dominant[1] * 1e-3) / 1e9
+    work = stage_work(cfg, split)
+    kern = stage_kernels(cfg, split)
+    t_stage = {k: float(stage[:, i].mean()) for i, k in enumerate(STAGES)}
+    dom = max(STAGES[1:], key=lambda k: t_stage[k])
+    dbytes, dflops = work[dom]
+    if dflops > 0:
+        roof = {"bound": "tensor", "achieved": dflops / (t_stage[dom] * 1e-3) / 1e12, "peak": bf16,
+                "unit": "TFLOP/s", "alg_flops_per_launch": dflops}
+    else:
+        roof = {"bound": "hbm", "achieved": dbytes / (t_stage[dom] * 1e-3) / 1e9, "peak": hbm,
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["alg_bytes_per_launch"] = dbytes
     traffic = None
     if os.path.exists(PROFILE_TRAFFIC):
         with open(PROFILE_TRAFFIC) as f:
             tr = json.load(f)
-        rec = tr.get(f"{cfg.name}:{dominant[0]}")
+        rec = tr.get(f"{cfg.name}:{dom}")
         if rec and rec.get("source_hash") == kernel_source_hash():
             traffic = rec["bytes_per_launch"]
+    roof["traffic"] = traffic
+    roof = {"kernel": kern[dom], "stage": dom, "peak_kind": peak_kind, **roof}
+    step_bytes = sum(b for b, _ in work.values())
+    per_expert = 2 * per_matrix_bytes(cfg.F, cfg.H) + per_matrix_bytes(cfg.H, cfg.F)
+    n_active = split["n_small"] + split["n_large"]
 
     if rank == 0:
         line = {
@@ -299,19 +359,16 @@ def main():
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "F": cfg.F, "K": cfg.K,
-                       "gs": 64, "distinct_experts": n_active, "parallelism": f"replicas x{world}",
+                       "gs": 64, "distinct_experts": n_active, "experts_tensor_core": split["n_large"],
+                       "parallelism": f"replicas x{world}",
                        "l2": f"{L2_FLUSH_BYTES >> 20} MiB flush between steps; touched weights "
-                             f"{n_active * 21233664 / 1e9:.2f} GB/step > L2"},
-            "hbm_gbs_step": ab["step"] / (ms * 1e-3) / 1e9,
-            "hbm_frac_of_8tbs": ab["step"] / (ms * 1e-3) / 8e12,
-            "stage_ms": {"route_rowmap": float(stage[:, 0].mean()), "gate_up": t_gu, "down": t_dn},
-            "roofline": {"kernel": f"gq4_skinny_kernel ({dominant[0]})", "bound": "hbm",
-                         "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": traffic,
-                         "alg_bytes_per_launch": ab[dominant[0]]},
+                             f"{n_active * per_expert / 1e9:.2f} GB/step"},
+            "hbm_gbs_step": step_bytes / (ms * 1e-3) / 1e9,
+            "stage_ms": t_stage,
+            "roofline": roof,
             "e2e": {"value": world * cfg.T / (e2e * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_h.nbytes + lg_h.nbytes, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches_per_step(cfg, split) * args.steps,
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline and world == 1:

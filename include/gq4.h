@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define GQ4_ABI_VERSION 1u
+#define GQ4_ABI_VERSION 2u
 
 typedef struct CUstream_st *gq4_stream_t; /* binary-compatible with cudaStream_t */
 typedef struct CUevent_st *gq4_event_t;   /* binary-compatible with cudaEvent_t */
@@ -176,13 +176,24 @@ gq4_status gq4_rowmap(const int32_t *idx, int64_t T, int32_t K, int32_t E, int32
  *   Wg, Wu: E stacked [F][H]; Wd: E stacked [H][F]; logits device f32 [T][E];
  *   x device bf16 [T][H]; y device f32 [T][H] (overwritten); ws device workspace of
  *   moe_expert_ffn_workspace_bytes(T, E, K, H, F) bytes; 1 <= K <= E <= 1024.
+ * Experts are split by their row count: with T >= GQ4_MOE_LARGE_MIN_ROWS, H % 128 == 0,
+ * F % 64 == 0 and expert strides that are whole rows, an expert with at least
+ * GQ4_MOE_LARGE_MIN_ROWS rows runs on the tensor-core kernels, the others (and every
+ * expert otherwise) on the decode kernels.  The split changes speed, not results
+ * beyond rounding.
  * Data-dependent errors (non-finite logits) are reported through the workspace status
  * word: read it with moe_expert_ffn_status.  The order in which the K slot
  * contributions are added into y is not fixed (float atomics); results agree within
  * rounding.
- *   stage_events: NULL, or 4 CUDA events (created by the caller) recorded on `stream`
- *   at the start, after the router and row map, after gate+up and after down, so a
- *   caller can time the stages with cudaEventElapsedTime. */
+ *   stage_events: NULL, or GQ4_MOE_STAGE_EVENTS (6) CUDA events (created by the caller)
+ *   recorded on `stream` at: [0] the start, [1] after the router and row map, [2] after
+ *   gate+up of the experts with few rows (decode kernels), [3] after gate+up of the
+ *   experts with many rows (row gather + tensor-core kernel), [4] after down of the
+ *   experts with few rows, [5] after down of the experts with many rows.  Where a stage
+ *   launches nothing its two events are recorded back to back.  A caller times the
+ *   stages with cudaEventElapsedTime. */
+#define GQ4_MOE_STAGE_EVENTS 6
+#define GQ4_MOE_LARGE_MIN_ROWS 24
 size_t moe_expert_ffn_workspace_bytes(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F);
 gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_tensor *Wd,
                           const float *logits, const void *x, gq4_dtype xdt, int64_t T,

@@ -151,7 +151,7 @@ struct MoeLayout {
 
 // Experts with at least this many rows go to the tensor-core (tcgen05) kernels, the
 // others to the decode kernels.
-constexpr int kLargeMin = 24;
+constexpr int kLargeMin = GQ4_MOE_LARGE_MIN_ROWS;
 
 inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -632,6 +632,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     st = band ? launch_band<kMoeGateUp>(pg, small_cols, max_active * ((pg.row_tiles + 7) / 8), status, s)
               : launch_skinny<kMoeGateUp>(pg, small_cols, false, max_active * pg.row_tiles, s);
     if (st != GQ4_OK) return st;
+    mark(2);
 
     // experts with many rows: gathered activations, tensor-core gate+up and down
     CUtensorMap tm_g, tm_u, tm_d, tm_x[4], tm_h[4];
@@ -667,7 +668,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
         st = launch_tc<0>(tm_g, tm_u, tm_x, tg, max_large * tg.m_tiles, s);
         if (st != GQ4_OK) return st;
     }
-    mark(2);
+    mark(3);
 
     SkinnyParams pd = p;
     pd.w0 = Wd->w; pd.s0 = Wd->s;
@@ -679,6 +680,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     st = band ? launch_band<kMoeDown>(pd, small_cols, max_active * ((pd.row_tiles + 7) / 8), status, s)
               : launch_skinny<kMoeDown>(pd, small_cols, false, max_active * pd.row_tiles, s);
     if (st != GQ4_OK) return st;
+    mark(4);
     if (tc) {
         const int max_large = std::max(1, std::min<int>(E, (int)(T * K / kLargeMin)));
         TcParams td = tp;
@@ -687,7 +689,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
         td.estride_rows = (int)(Wd->expert_stride_w / (F / 2));
         st = launch_tc<1>(tm_d, tm_d, tm_h, td, max_large * td.m_tiles, s);
     }
-    mark(3);
+    mark(5);
     return st;
 }
 

@@ -16,7 +16,9 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgq4.so")
-ABI_VERSION = 1
+ABI_VERSION = 2
+MOE_STAGE_EVENTS = 6
+MOE_LARGE_MIN_ROWS = 24  # GQ4_MOE_LARGE_MIN_ROWS
 
 OK, ERR_NULL, ERR_ALIGN, ERR_SHAPE, ERR_UNSUPPORTED, ERR_ALIAS, ERR_WORKSPACE, ERR_CUDA, \
     ERR_TIMEOUT, ERR_NONFINITE_LOGIT = range(10)
@@ -291,8 +293,9 @@ def moe_expert_ffn(Wg: Tensor, Wu: Tensor, Wd: Tensor, logits: torch.Tensor, x: 
                    stage_events=None):
     """y [T][H] f32 for one routed-expert FFN layer (x bf16 [T][H], logits f32 [T][E]).
 
-    stage_events: optional 4 torch.cuda.Event(enable_timing=True) recorded at the start,
-    after routing, after gate+up and after down."""
+    stage_events: optional 6 torch.cuda.Event(enable_timing=True) recorded at the start,
+    after routing, after gate+up of the experts with few rows, after gate+up of those
+    with many rows, after down of the few-row experts and after down of the others."""
     T, H = x.shape
     E = logits.shape[1]
     F = Wg.out
@@ -303,7 +306,9 @@ def moe_expert_ffn(Wg: Tensor, Wu: Tensor, Wd: Tensor, logits: torch.Tensor, x: 
     _need_cuda(x, logits, y)
     ev = None
     if stage_events is not None:
-        ev = (ctypes.c_void_p * 4)(*[e.cuda_event for e in stage_events])
+        if len(stage_events) != MOE_STAGE_EVENTS:
+            raise ValueError(f"stage_events: {MOE_STAGE_EVENTS} events expected")
+        ev = (ctypes.c_void_p * MOE_STAGE_EVENTS)(*[e.cuda_event for e in stage_events])
     _check(_lib.moe_expert_ffn(Wg.ref(), Wu.ref(), Wd.ref(), logits.data_ptr(), x.data_ptr(), _xdt(x),
                                T, E, K, y.data_ptr(), ws.buf.data_ptr(), ws.nbytes, ev, _stream(stream)),
            "moe_expert_ffn")
