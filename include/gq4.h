@@ -211,6 +211,33 @@ gq4_status moe_expert_ffn_status(const void *ws, size_t ws_bytes, int64_t T, int
                                  int32_t K, int64_t H, int64_t F, gq4_stream_t stream,
                                  int32_t *status);
 
+/* moe_expert_ffn_noalloc: the same layer as moe_expert_ffn, for callers that cannot
+ * allocate device memory -- a plug-in whose host program owns every device allocation
+ * and hands it only the tensors, or a decode loop that must not call cudaMalloc because
+ * cudaMalloc can synchronise the device.  It has no counterpart on the source pages: it
+ * exists only so that such callers need no workspace.
+ *   Instead of a caller workspace it uses one library-owned device array of
+ *   GQ4_NOALLOC_SCRATCH_BYTES (16 MiB), which every GPU that loads this library holds
+ *   until the process exits.  A shape whose workspace
+ *   (moe_expert_ffn_workspace_bytes(T, E, K, H, F)) exceeds that returns
+ *   GQ4_ERR_WORKSPACE before anything is launched; 16 MiB covers decode batches up to
+ *   about 120 tokens at H = 6144, F = 2048, K = 8, E = 256.
+ *   Arguments as for moe_expert_ffn (no stage events); status_out is NULL or a 16-byte
+ *   aligned device int32 that receives the data-error status word of this call
+ *   (GQ4_ERR_NONFINITE_LOGIT ...), copied on `stream` after the layer.
+ *   The first call on a device looks up that device's address of the array (with the
+ *   device current); make that first call before any stream capture.  The call itself
+ *   calls no cudaMalloc, cudaFree or other allocating routine.
+ *   Every call, on every stream, shares the one array per device and it keeps the last
+ *   call's contents; the call clears what must start at zero (the status word).  Calls
+ *   that overlap on the GPU -- on two streams, or from two host threads -- race on the
+ *   array and corrupt each other's results: serialise them. */
+#define GQ4_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+gq4_status moe_expert_ffn_noalloc(const gq4_tensor *Wg, const gq4_tensor *Wu,
+                                  const gq4_tensor *Wd, const float *logits, const void *x,
+                                  gq4_dtype xdt, int64_t T, int32_t E, int32_t K, float *y,
+                                  int32_t *status_out, gq4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -694,3 +694,61 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
 }
 
 }  // extern "C"
+
+// ---- allocation-free variant of moe_expert_ffn ------------------------------------------
+// For callers that may not allocate device memory, the workspace lives in this one
+// library-owned array.  In host code its name stands for a host-side shadow, not for
+// device memory: the device address is looked up per device with cudaGetSymbolAddress
+// and only that address is handed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GQ4_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[kNoallocMaxDevices];  // device address of the array, per device
+
+// Device address of the array on the current device (looked up on first use).
+gq4_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQ4_ERR_CUDA;
+    if (dev < 0 || dev >= kNoallocMaxDevices) return GQ4_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ4_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return GQ4_OK;
+}
+}  // namespace
+
+extern "C" gq4_status moe_expert_ffn_noalloc(const gq4_tensor *Wg, const gq4_tensor *Wu,
+                                             const gq4_tensor *Wd, const float *logits,
+                                             const void *x, gq4_dtype xdt, int64_t T, int32_t E,
+                                             int32_t K, float *y, int32_t *status_out,
+                                             gq4_stream_t stream) {
+    if (!Wg || !Wu || !Wd) return GQ4_ERR_NULL;
+    if (T < 1 || E < 1 || K < 1 || K > E || Wg->in < 1 || Wg->out < 1) return GQ4_ERR_SHAPE;
+    if (status_out && !aligned16(status_out)) return GQ4_ERR_ALIGN;
+    const MoeLayout L = moe_layout(T, E, K, Wg->in, Wg->out);
+    if (L.total > GQ4_NOALLOC_SCRATCH_BYTES) return GQ4_ERR_WORKSPACE;
+    void *ws = nullptr;
+    gq4_status st = noalloc_scratch(&ws);
+    if (st != GQ4_OK) return st;
+    if (!logits || !x || !y) return GQ4_ERR_NULL;
+    if (status_out) {
+        const Range sr = rng(status_out, 4);
+        if (overlap(sr, rng(y, (size_t)T * Wg->in * 4)) || overlap(sr, rng(logits, (size_t)T * E * 4)) ||
+            overlap(sr, rng(x, (size_t)T * Wg->in * 2)))
+            return GQ4_ERR_ALIAS;
+    }
+    // moe_expert_ffn validates everything else and clears the status word itself
+    st = moe_expert_ffn(Wg, Wu, Wd, logits, x, xdt, T, E, K, y, ws, GQ4_NOALLOC_SCRATCH_BYTES, nullptr,
+                        stream);
+    if (st != GQ4_OK || !status_out) return st;
+    if (cudaMemcpyAsync(status_out, (const char *)ws + L.status, 4, cudaMemcpyDeviceToDevice, S(stream)) !=
+        cudaSuccess)
+        return GQ4_ERR_CUDA;
+    return GQ4_OK;
+}

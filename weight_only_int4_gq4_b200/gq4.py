@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libgq4.so")
 ABI_VERSION = 2
 MOE_STAGE_EVENTS = 6
 MOE_LARGE_MIN_ROWS = 24  # GQ4_MOE_LARGE_MIN_ROWS
+NOALLOC_SCRATCH_BYTES = 16 << 20  # GQ4_NOALLOC_SCRATCH_BYTES
 
 OK, ERR_NULL, ERR_ALIGN, ERR_SHAPE, ERR_UNSUPPORTED, ERR_ALIAS, ERR_WORKSPACE, ERR_CUDA, \
     ERR_TIMEOUT, ERR_NONFINITE_LOGIT = range(10)
@@ -65,6 +66,8 @@ _SIGS = {
                                ctypes.c_int),
     "moe_expert_ffn_status": ([_P, _SZ, _I64, _I32, _I32, _I64, _I64, _P, ctypes.POINTER(_I32)],
                               ctypes.c_int),
+    "moe_expert_ffn_noalloc": ([_TP, _TP, _TP, _P, _P, ctypes.c_int, _I64, _I32, _I32, _P, _P, _P],
+                               ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -313,3 +316,20 @@ def moe_expert_ffn(Wg: Tensor, Wu: Tensor, Wd: Tensor, logits: torch.Tensor, x: 
                                T, E, K, y.data_ptr(), ws.buf.data_ptr(), ws.nbytes, ev, _stream(stream)),
            "moe_expert_ffn")
     return y, ws
+
+
+def moe_expert_ffn_noalloc(Wg: Tensor, Wu: Tensor, Wd: Tensor, logits: torch.Tensor, x: torch.Tensor,
+                           K: int, y: torch.Tensor, status_out: torch.Tensor | None = None, stream=None):
+    """moe_expert_ffn without a workspace, for callers that cannot allocate device memory.
+
+    The library's own device array (NOALLOC_SCRATCH_BYTES per GPU) replaces the
+    workspace; y (and status_out, a device int32 tensor of at least one element, if given)
+    are the caller's.  Calls that overlap on the GPU share that array and race: serialise
+    them."""
+    T, H = x.shape
+    E = logits.shape[1]
+    _need_cuda(x, logits, y, status_out)
+    _check(_lib.moe_expert_ffn_noalloc(Wg.ref(), Wu.ref(), Wd.ref(), logits.data_ptr(), x.data_ptr(),
+                                       _xdt(x), T, E, K, y.data_ptr(), _ptr(status_out), _stream(stream)),
+           "moe_expert_ffn_noalloc")
+    return y
