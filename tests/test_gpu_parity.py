@@ -41,6 +41,10 @@ MV_CASES = [
     (16, 64, 1, "bf16"), (50, 256, 1, "bf16"), (200, 640, 3, "f32"), (33, 1024, 9, "bf16"),
     (64, 512, 20, "bf16"), (16, 128, 40, "bf16"), (100, 4096, 1, "f32"), (7, 192, 2, "f32"),
     (1000, 1536, 5, "bf16"), (24, 64, 11, "f32"),
+    # TMA-fed decode kernel: 128- and 64-row bands, 1..4 n-tiles, two column passes,
+    # ragged row tails, a single column over many bands
+    (300, 2048, 32, "bf16"), (130, 768, 17, "bf16"), (520, 1024, 24, "bf16"), (96, 256, 33, "bf16"),
+    (9600, 256, 1, "bf16"), (9500, 512, 2, "bf16"),
 ]
 
 
@@ -242,7 +246,11 @@ def _toy(T, E, K, H=128, F=128, seed=3, **kw):
                                        # tensor-core path (experts with >= 24 rows), mixed with
                                        # the decode path, multi-pass experts (> 192 rows)
                                        (64, 4, 2, 256, 128), (40, 8, 4, 384, 192), (300, 2, 1, 128, 64),
-                                       (500, 2, 2, 128, 128), (48, 4, 2, 192, 128), (130, 6, 3, 512, 256)])
+                                       (500, 2, 2, 128, 128), (48, 4, 2, 192, 128), (130, 6, 3, 512, 256),
+                                       # TMA-fed decode kernel for gate+up and down (H, F multiples
+                                       # of 256), alone and beside the tensor-core path
+                                       (12, 16, 4, 256, 256), (30, 8, 8, 512, 256), (20, 64, 8, 256, 512),
+                                       (9, 4, 4, 768, 1280)])
 def test_moe_small_full_oracle(T, E, K, H, F):
     s = MoESet(_toy(T, E, K, H, F))
     y, ws = s.run()

@@ -13,6 +13,7 @@
 #include "gq4_common.cuh"
 #include "gq4_route.cuh"
 #include "gq4_skinny.cuh"
+#include "gq4_stream.cuh"
 #include "gq4_tc.cuh"
 
 using namespace gq4;
@@ -301,6 +302,95 @@ bool make_act_maps(CUtensorMap (&m)[4], const void *base, uint64_t cols, uint64_
     return true;
 }
 
+// ---- TMA-fed decode kernel (gq4_stream.cuh) ------------------------------------------
+// The matrices (or expert stacks) it reads: packed weights and scales of matrix 0 and,
+// for gate+up, matrix 1, with their expert strides in rows.
+struct StreamMats {
+    const uint8_t *w0, *w1;
+    const float *s0, *s1;
+    int64_t n_experts, wrows, srows;  // expert strides in rows of the packed / scale arrays
+};
+
+// The kernel streams whole four-group stages and addresses experts by row: bf16
+// activations, ng % 4 == 0, and expert strides that are whole rows.
+bool stream_usable(const gq4_tensor *t) {
+    if (t->ng % kStGroups) return false;
+    if (t->n_experts > 1 && (t->expert_stride_w % (t->in / 2) || t->expert_stride_s % t->ng)) return false;
+    return true;
+}
+
+StreamMats stream_mats(const gq4_tensor *t0, const gq4_tensor *t1) {
+    StreamMats m{};
+    m.w0 = t0->w; m.s0 = t0->s;
+    m.w1 = t1 ? t1->w : t0->w; m.s1 = t1 ? t1->s : t0->s;
+    m.n_experts = t0->n_experts;
+    m.wrows = t0->n_experts > 1 ? t0->expert_stride_w / (t0->in / 2) : t0->out;
+    m.srows = t0->n_experts > 1 ? t0->expert_stride_s / t0->ng : t0->out;
+    return m;
+}
+
+template <int MODE, int NT, int RW>
+gq4_status launch_stream_k(const StreamMats &m, const SkinnyParams &p, int units_upper, int32_t *status,
+                           cudaStream_t st) {
+    constexpr int PAIR = ModeTraits<MODE>::kPair;
+    constexpr int BR = 16 * RW;
+    auto kern = gq4_stream_kernel<MODE, NT, RW>;
+    StreamArgs a{};
+    a.stage_bytes = stream_stage_bytes(PAIR, BR, std::min(kStMaxCols, NT * 8));
+    const int budget = (int)kMaxSmem - stream_xch_bytes(RW, NT) - 16 - 1024;
+    a.nstages = std::min(8, budget / (a.stage_bytes + 16));
+    if (a.nstages < 2) return GQ4_ERR_UNSUPPORTED;
+    a.wrows = (int)m.wrows;
+    a.srows = (int)m.srows;
+    a.status = status;
+    const size_t smem = stream_smem_bytes(a.nstages, a.stage_bytes, RW, NT);
+    if (smem > kMaxSmem) return GQ4_ERR_UNSUPPORTED;
+    CUtensorMap tm[4];
+    const uint64_t rows_w = (uint64_t)(m.n_experts - 1) * m.wrows + p.O;
+    const uint64_t rows_s = (uint64_t)(m.n_experts - 1) * m.srows + p.O;
+    for (int i = 0; i < 2; ++i) {
+        if (!make_tmap_2d(&tm[i], i ? m.w1 : m.w0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.I / 2, rows_w, 128, BR,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_2d(&tm[2 + i], i ? m.s1 : m.s0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.ng, rows_s,
+                          kStGroups, BR, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return GQ4_ERR_CUDA;
+    }
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GQ4_ERR_CUDA;
+    const int grid = std::max(1, std::min(units_upper, sm_count()));
+    kern<<<grid, kStThreads, smem, st>>>(tm[0], tm[1], tm[2], tm[3], p, a);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
+// Band height: the tallest whose unit count gives every SM at least two bands (gate+up:
+// 128 or 64 rows of each matrix; down and plain matvec: 256, 128 or 64 rows), else the
+// smallest.  The n-tile count covers the columns of one pass.  `mats` = matrices
+// (experts) the call may touch.
+template <int MODE, int NT>
+gq4_status launch_stream_nt(const StreamMats &m, const SkinnyParams &p, int mats, int32_t *status,
+                            cudaStream_t st) {
+    auto units = [&](int br) { return mats * ((p.O + br - 1) / br); };
+    const int want = 2 * sm_count();
+    if constexpr (ModeTraits<MODE>::kPair == 2) {
+        if (units(128) >= want) return launch_stream_k<MODE, NT, 8>(m, p, units(128), status, st);
+        return launch_stream_k<MODE, NT, 4>(m, p, units(64), status, st);
+    } else {
+        if (units(256) >= want) return launch_stream_k<MODE, NT, 16>(m, p, units(256), status, st);
+        if (units(128) >= want) return launch_stream_k<MODE, NT, 8>(m, p, units(128), status, st);
+        return launch_stream_k<MODE, NT, 4>(m, p, units(64), status, st);
+    }
+}
+
+template <int MODE>
+gq4_status launch_stream(const StreamMats &m, const SkinnyParams &p, int max_cols, int mats, int32_t *status,
+                         cudaStream_t st) {
+    const int c = std::min(max_cols, kStMaxCols);
+    if (c <= 8) return launch_stream_nt<MODE, 1>(m, p, mats, status, st);
+    if (c <= 16) return launch_stream_nt<MODE, 2>(m, p, mats, status, st);
+    if (c <= 24) return launch_stream_nt<MODE, 3>(m, p, mats, status, st);
+    return launch_stream_nt<MODE, 4>(m, p, mats, status, st);
+}
+
 template <int MODE>
 gq4_status launch_tc(const CUtensorMap &w0, const CUtensorMap &w1, const CUtensorMap (&x)[4],
                      const TcParams &p, int units_upper, cudaStream_t st) {
@@ -430,6 +520,8 @@ gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.y = y;
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    if (xdt == GQ4_BF16 && stream_usable(W) && (n_tok >= kBandMinCols || (W->out + 63) / 64 >= sm_count()))
+        return launch_stream<kMatvec>(stream_mats(W, nullptr), p, cols, 1, nullptr, S(stream));
     if (xdt == GQ4_BF16 && n_tok >= kBandMinCols)
         return launch_band<kMatvec>(p, cols, (p.row_tiles + 7) / 8, nullptr, S(stream));
     return launch_skinny<kMatvec>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
@@ -459,6 +551,9 @@ gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const vo
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.h = h;
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    if (xdt == GQ4_BF16 && stream_usable(Wg) && stream_usable(Wu) &&
+        (n_tok >= kBandMinCols || (Wg->out + 63) / 64 >= sm_count()))
+        return launch_stream<kGateUp>(stream_mats(Wg, Wu), p, cols, 1, nullptr, S(stream));
     if (xdt == GQ4_BF16 && n_tok >= kBandMinCols)
         return launch_band<kGateUp>(p, cols, (p.row_tiles + 7) / 8, nullptr, S(stream));
     return launch_skinny<kGateUp>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
@@ -629,8 +724,12 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     const int small_cols = (int)std::min<int64_t>(max_cols, tc ? kLargeMin - 1 : max_cols);
     const bool band = small_cols >= kBandMinCols;
     int32_t *status = at<int32_t>(ws, L.status);
-    st = band ? launch_band<kMoeGateUp>(pg, small_cols, max_active * ((pg.row_tiles + 7) / 8), status, s)
-              : launch_skinny<kMoeGateUp>(pg, small_cols, false, max_active * pg.row_tiles, s);
+    const bool stream_gu = stream_usable(Wg) && stream_usable(Wu) && Wu->expert_stride_s == Wg->expert_stride_s;
+    if (stream_gu)
+        st = launch_stream<kMoeGateUp>(stream_mats(Wg, Wu), pg, small_cols, max_active, status, s);
+    else
+        st = band ? launch_band<kMoeGateUp>(pg, small_cols, max_active * ((pg.row_tiles + 7) / 8), status, s)
+                  : launch_skinny<kMoeGateUp>(pg, small_cols, false, max_active * pg.row_tiles, s);
     if (st != GQ4_OK) return st;
     mark(2);
 
@@ -677,8 +776,11 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     pd.row_tiles = (int)((H + 15) / 16);
     pd.x = at<void>(ws, L.h); pd.xdt = 1; pd.n_tok = (int)T;
     pd.y = y;
-    st = band ? launch_band<kMoeDown>(pd, small_cols, max_active * ((pd.row_tiles + 7) / 8), status, s)
-              : launch_skinny<kMoeDown>(pd, small_cols, false, max_active * pd.row_tiles, s);
+    if (stream_usable(Wd))
+        st = launch_stream<kMoeDown>(stream_mats(Wd, nullptr), pd, small_cols, max_active, status, s);
+    else
+        st = band ? launch_band<kMoeDown>(pd, small_cols, max_active * ((pd.row_tiles + 7) / 8), status, s)
+                  : launch_skinny<kMoeDown>(pd, small_cols, false, max_active * pd.row_tiles, s);
     if (st != GQ4_OK) return st;
     mark(4);
     if (tc) {

@@ -1,0 +1,373 @@
+// gq4_stream.cuh -- TMA-fed decode kernel for grouped-int4 products with few activation
+// columns (1..32 per matrix or expert): the HBM-bound regime of the routed-expert FFN.
+//
+// What it computes (colibri PR #298, "cuda+engine: full fmt=4 (grouped int4 gs=64)
+// support"): y[c][o] = sum_g s[o][g] * sum_{k in group g} q[o][k] * x[c][k], the group
+// scale applied once per 64-wide group to an f32 partial, fp32 accumulation; for gate+up
+// h = bf16(silu(g) * u); for the MoE down projection a weighted scatter-add into y.
+//
+// Design (B200, HBM-bound):
+//  * A CTA (one per SM, persistent) owns a band of BR = 16*RW rows of one matrix or
+//    expert (for gate+up: BR gate rows and the same BR up rows) for all of K.
+//  * One producer warp streams the band through a ring of shared-memory stages, four
+//    64-wide groups per stage: the packed nibble tile of each matrix (BR rows x 128 B,
+//    one 2-D TMA copy, 128-byte swizzle), the f32 scales of those rows and groups (BR x
+//    16 B, one TMA copy) and the stage's 256 activations of every column (one bulk copy
+//    per column; the source address does the token gather).  Completion is an mbarrier
+//    with a transaction count; no thread spends instructions on weight addresses.
+//  * Sixteen consumer warps: RW row warps x KW = 16/RW k-warps.  A row warp owns 16 rows;
+//    its k-warps split the stage's (matrix, group) items (gate+up: one matrix each; down:
+//    256-row bands need no split).  Each item is one m16n8k16 tensor op chain per 8
+//    columns: the nibbles become exact bf16 integers (one lop3 + one bf16x2 fma per two
+//    weights), the f32 partial of the group is scaled by s[o][g] and added to the running
+//    sum.  The integer pipe is the scarce one (the nibble decode lives there), so every
+//    address, slot and phase is computed incrementally or once per warp.
+//  * At the end of a band the k-warps' sums are added in a fixed order through shared
+//    memory (deterministic) and the mode's epilogue runs.
+// Every wait is bounded (~2 s): on expiry GQ4_ERR_TIMEOUT is raised in the status word,
+// the other waits return at once, all warps still pass the same barriers, and the
+// producer lets its copies in flight land before the CTA leaves.
+#pragma once
+#include <cuda.h>
+
+#include "gq4_common.cuh"
+#include "gq4_skinny.cuh"
+#include "gq4_tc.cuh"
+
+namespace gq4 {
+
+constexpr int kStConsumerWarps = 16;
+constexpr int kStThreads = (kStConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kStMaxCols = 32;                            // columns per pass
+constexpr int kStXStride = 528;  // bytes per staged activation row: 256 bf16 + 16 B pad
+constexpr int kStGroups = 4;     // groups per stage (128 packed bytes per row)
+
+struct StreamArgs {
+    int nstages;       // ring depth
+    int stage_bytes;   // bytes per stage (multiple of 1024)
+    int wrows;         // rows per expert in the weight tensor maps
+    int srows;         // rows per expert in the scale tensor maps
+    int32_t *status;   // device status word (GQ4_ERR_TIMEOUT), may be NULL
+};
+
+__host__ __device__ inline int stream_stage_bytes(int pair, int br, int ncols) {
+    const int b = pair * br * 128 + pair * br * 16 + ncols * kStXStride;
+    return (b + 1023) & ~1023;
+}
+__host__ __device__ inline int stream_xch_bytes(int rw, int nt) {
+    return rw * (kStConsumerWarps / rw - 1) * nt * 4 * 32 * 4;
+}
+// ring + exchange buffer + 2 mbarriers per stage + abort flag + 1024 for alignment
+__host__ __device__ inline int stream_smem_bytes(int nstages, int stage_bytes, int rw, int nt) {
+    return nstages * stage_bytes + stream_xch_bytes(rw, nt) + 16 * nstages + 16 + 1024;
+}
+
+// Four bf16x2 pairs of one device word (nibble slots i and i+4 -> columns 2i, 2i+1).
+__device__ __forceinline__ void word_to_bf16x4(uint32_t v, uint32_t *r) {
+    r[0] = nib2_to_bf16x2(v);
+    r[1] = nib2_to_bf16x2(v >> 4);
+    r[2] = nib2_to_bf16x2(v >> 8);
+    r[3] = nib2_to_bf16x2(v >> 12);
+}
+
+// Bounded wait for the phase of `parity`; false once the CTA has aborted or ~2 s passed
+// (then GQ4_ERR_TIMEOUT is raised in *status when a status word was given).
+__device__ __forceinline__ bool st_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                        int32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if ((i & 7) == 0) {
+            if (*abort_flag) return false;
+            if (global_ns() - t0 > 2000000000ull) {
+                *abort_flag = 1;
+                if (status) atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void named_bar_consumers() {
+    asm volatile("bar.sync 1, %0;" ::"r"(kStConsumerWarps * 32) : "memory");
+}
+
+// The items of one stage for one consumer warp: groups GL0 .. GL0+IPW-1 of its matrix.
+//   a_row: its packed tile row R (and R+8 at +1024); s_row: the four scales of row R (row
+//   R+8 at +128); x_lane: the activation bytes this lane feeds for n-tile 0, group 0.
+// Columns past nc hold stale values: they only reach accumulator columns that are never
+// stored, so they need no zeroing.
+template <int NT, int NTA, int IPW, int GL0>
+__device__ __forceinline__ void stream_items_n(const uint8_t *a_row, const uint8_t *s_row, const uint8_t *x_lane,
+                                             const int (&aoff)[kStGroups], float (&acc)[NT][4]) {
+    const float4 sva = *(const float4 *)s_row;
+    const float4 svb = *(const float4 *)(s_row + 8 * 16);
+    #pragma unroll
+    for (int q = 0; q < IPW; ++q) {
+        const int gl = GL0 + q;
+        const uint2 wa = *(const uint2 *)(a_row + aoff[gl]);
+        const uint2 wb = *(const uint2 *)(a_row + 8 * 128 + aoff[gl]);
+        const float sa = gl == 0 ? sva.x : gl == 1 ? sva.y : gl == 2 ? sva.z : sva.w;
+        const float sb = gl == 0 ? svb.x : gl == 1 ? svb.y : gl == 2 ? svb.z : svb.w;
+        const uint64_t ssa = splat2(sa), ssb = splat2(sb);
+        uint32_t ra[8], rb[8];
+        word_to_bf16x4(wa.x, ra);
+        word_to_bf16x4(wa.y, ra + 4);
+        word_to_bf16x4(wb.x, rb);
+        word_to_bf16x4(wb.y, rb + 4);
+        #pragma unroll
+        for (int n = 0; n < NTA; ++n) {
+            const uint4 *src = (const uint4 *)(x_lane + n * 8 * kStXStride + gl * 128);
+            const uint4 b0 = src[0], b1 = src[1];
+            const uint32_t bf[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t af[4] = {ra[2 * j], rb[2 * j], ra[2 * j + 1], rb[2 * j + 1]};
+                mma_bf16_16816(d, af, bf[2 * j], bf[2 * j + 1], d);
+            }
+            fma2(acc[n][0], acc[n][1], d[0], d[1], ssa);
+            fma2(acc[n][2], acc[n][3], d[2], d[3], ssb);
+        }
+    }
+}
+
+template <int NT, int IPW, int GL0>
+__device__ __forceinline__ void stream_items(const uint8_t *a_row, const uint8_t *s_row, const uint8_t *x_lane,
+                                             const int (&aoff)[kStGroups], int nc, float (&acc)[NT][4]) {
+    if (NT >= 4 && nc > 24) stream_items_n<NT, (NT >= 4 ? 4 : 1), IPW, GL0>(a_row, s_row, x_lane, aoff, acc);
+    else if (NT >= 3 && nc > 16) stream_items_n<NT, (NT >= 3 ? 3 : 1), IPW, GL0>(a_row, s_row, x_lane, aoff, acc);
+    else if (NT >= 2 && nc > 8) stream_items_n<NT, (NT >= 2 ? 2 : 1), IPW, GL0>(a_row, s_row, x_lane, aoff, acc);
+    else stream_items_n<NT, 1, IPW, GL0>(a_row, s_row, x_lane, aoff, acc);
+}
+
+template <int MODE, int NT, int RW>
+__global__ void __launch_bounds__(kStThreads, 1)
+gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
+                  const __grid_constant__ CUtensorMap tm_s0, const __grid_constant__ CUtensorMap tm_s1,
+                  const SkinnyParams p, const StreamArgs a) {
+    using TR = ModeTraits<MODE>;
+    constexpr int PAIR = TR::kPair;
+    constexpr int BR = 16 * RW;
+    constexpr int KW = kStConsumerWarps / RW;   // k-warps per row warp
+    constexpr int IPW = kStGroups * PAIR / KW;  // (matrix, group) items per warp per stage
+    constexpr int KPM = KW / PAIR;              // k-warps per matrix
+    static_assert(IPW >= 1 && IPW <= kStGroups && KW % PAIR == 0, "item split");
+    constexpr int WBOX = BR * 128, SBOX = BR * 16;
+    constexpr int XOFF = PAIR * (WBOX + SBOX);
+    constexpr int PW = NT * 8 < kStMaxCols ? NT * 8 : kStMaxCols;  // columns per pass (x rows a stage holds)
+
+    extern __shared__ uint8_t st_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)st_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(sm);
+    const int NS = a.nstages, SB = a.stage_bytes;
+    float *xch = (float *)(sm + NS * SB);
+    const uint32_t bar0 = sbase + NS * SB + stream_xch_bytes(RW, NT);
+    auto full_bar = [&](int s) { return bar0 + 8 * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8 * (NS + s); };
+    volatile int *abort_flag = (volatile int *)(sm + NS * SB + stream_xch_bytes(RW, NT) + 16 * NS);
+    int32_t *status = a.status;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), kStConsumerWarps);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (MODE == kMoeGateUp && p.zero_ptr) {  // y is accumulated into by the down kernel
+        float4 *z = (float4 *)p.zero_ptr;
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_n / 4;
+             i += (int64_t)gridDim.x * blockDim.x)
+            z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+
+    const int bands = (p.O + BR - 1) / BR;
+    const int n_units = TR::kMoe ? (*p.n_active) * bands : bands;
+    const int nst = p.ng / kStGroups;  // stages per pass
+
+    uint32_t issued = 0;  // stages the producer warp issued
+    if (warp == kStConsumerWarps) {
+        // ------------------------------------------------------------ producer warp
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            int e = 0, band = u, row0 = 0, cols = p.n_tok;
+            if (TR::kMoe) {
+                const int ai = u / bands;
+                band = u - ai * bands;
+                e = p.active[ai];
+                row0 = p.offs[e];
+                cols = p.cnt[e];
+            }
+            const int wrow = e * a.wrows + band * BR, srow = e * a.srows + band * BR;
+            for (int c0 = 0; c0 < cols; c0 += PW) {
+                const int nc = min(PW, cols - c0);
+                const uint16_t *xrow = nullptr;  // this lane's activation row
+                if (lane < nc) {
+                    if (MODE == kMoeGateUp)
+                        xrow = (const uint16_t *)p.x + (int64_t)p.row_tok[row0 + c0 + lane] * p.I;
+                    else if (MODE == kMoeDown)
+                        xrow = (const uint16_t *)p.x + (int64_t)(row0 + c0 + lane) * p.I;
+                    else
+                        xrow = (const uint16_t *)p.x + (int64_t)(c0 + lane) * p.I;
+                }
+                const uint32_t tx = (uint32_t)(XOFF + nc * 512);
+                for (int k = 0; k < nst; ++k) {
+                    if (ok && lane == 0) ok = st_wait(empty_bar(s), ph ^ 1u, abort_flag, status) && !*abort_flag;
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (ok) {
+                        const uint32_t stg = sbase + s * SB;
+                        if (lane == 0) {
+                            mbar_expect_tx(full_bar(s), tx);
+                            tma_load_2d(stg, &tm_w0, k * 128, wrow, full_bar(s));
+                            if (PAIR == 2) tma_load_2d(stg + WBOX, &tm_w1, k * 128, wrow, full_bar(s));
+                            tma_load_2d(stg + PAIR * WBOX, &tm_s0, k * kStGroups, srow, full_bar(s));
+                            if (PAIR == 2)
+                                tma_load_2d(stg + PAIR * WBOX + SBOX, &tm_s1, k * kStGroups, srow, full_bar(s));
+                        }
+                        __syncwarp();
+                        if (lane < nc)
+                            bulk_g2s(stg + XOFF + lane * kStXStride, xrow + k * 256, 512u, full_bar(s));
+                        ++issued;
+                    }
+                    if (++s == NS) { s = 0; ph ^= 1u; }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ consumer warps
+        const int g = lane >> 2, t = lane & 3;
+        const int rw = warp % RW, kw = warp / RW;
+        const int m = (kw * IPW) / kStGroups;    // matrix of this warp's items
+        const int gl0 = (kw * IPW) % kStGroups;  // its first group in a stage
+        const int R = 16 * rw + g;               // band row of accumulator slots 0,1 (2,3: R+8)
+        // 128B swizzle: 16-byte chunk c of tile row r sits at chunk c ^ (r & 7), and
+        // (R & 7) == ((R + 8) & 7) == g; lane t reads bytes 8t..8t+7 of each group
+        int aoff[kStGroups];
+        #pragma unroll
+        for (int gl = 0; gl < kStGroups; ++gl) aoff[gl] = (((2 * gl + (t >> 1)) ^ g) << 4) | ((t & 1) << 3);
+        const int a_base = m * WBOX + R * 128;
+        const int s_base = PAIR * WBOX + m * SBOX + R * 16;
+        const int x_base = XOFF + g * kStXStride + t * 32;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            int e = 0, band = u, row0 = 0, cols = p.n_tok;
+            if (TR::kMoe) {
+                const int ai = u / bands;
+                band = u - ai * bands;
+                e = p.active[ai];
+                row0 = p.offs[e];
+                cols = p.cnt[e];
+            }
+            for (int c0 = 0; c0 < cols; c0 += PW) {
+                const int nc = min(PW, cols - c0);
+                float acc[NT][4];
+                #pragma unroll
+                for (int n = 0; n < NT; ++n)
+                    #pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+
+                for (int k = 0; k < nst; ++k) {
+                    if (st_wait(full_bar(s), ph, abort_flag, status)) {
+                        const uint8_t *stg = sm + s * SB;
+                        const uint8_t *ar = stg + a_base, *sr = stg + s_base, *xl = stg + x_base;
+                        if constexpr (IPW == 4) {
+                            stream_items<NT, 4, 0>(ar, sr, xl, aoff, nc, acc);
+                        } else if constexpr (IPW == 2) {
+                            if (gl0 == 0) stream_items<NT, 2, 0>(ar, sr, xl, aoff, nc, acc);
+                            else stream_items<NT, 2, 2>(ar, sr, xl, aoff, nc, acc);
+                        } else {
+                            if (gl0 == 0) stream_items<NT, 1, 0>(ar, sr, xl, aoff, nc, acc);
+                            else if (gl0 == 1) stream_items<NT, 1, 1>(ar, sr, xl, aoff, nc, acc);
+                            else if (gl0 == 2) stream_items<NT, 1, 2>(ar, sr, xl, aoff, nc, acc);
+                            else stream_items<NT, 1, 3>(ar, sr, xl, aoff, nc, acc);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty_bar(s));
+                    if (++s == NS) { s = 0; ph ^= 1u; }
+                }
+
+                // ---- combine the k-warps (fixed order) and run the epilogue
+                float v0[NT][4], v1[NT][4];
+                if constexpr (KW > 1) {
+                    if (kw != 0) {
+                        float *dst = xch + (rw * (KW - 1) + kw - 1) * NT * 4 * 32 + lane;
+                        #pragma unroll
+                        for (int n = 0; n < NT; ++n)
+                            #pragma unroll
+                            for (int i = 0; i < 4; ++i) dst[(n * 4 + i) * 32] = acc[n][i];
+                    }
+                    named_bar_consumers();
+                    if (kw == 0) {
+                        #pragma unroll
+                        for (int n = 0; n < NT; ++n)
+                            #pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                float s0 = acc[n][i], s1 = 0.f;
+                                #pragma unroll
+                                for (int w = 1; w < KW; ++w) {
+                                    const float v = xch[((rw * (KW - 1) + w - 1) * NT * 4 + n * 4 + i) * 32 + lane];
+                                    if (w < KPM) s0 += v; else s1 += v;
+                                }
+                                v0[n][i] = s0;
+                                v1[n][i] = s1;
+                            }
+                    }
+                    named_bar_consumers();  // the exchange buffer may be rewritten
+                } else {
+                    #pragma unroll
+                    for (int n = 0; n < NT; ++n)
+                        #pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            v0[n][i] = acc[n][i];
+                            v1[n][i] = 0.f;
+                        }
+                }
+                if (kw == 0 && !*abort_flag) {
+                    #pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        #pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int cl = n * 8 + 2 * t + (i & 1);
+                            const int o = band * BR + R + ((i >> 1) << 3);
+                            if (cl >= nc || o >= p.O) continue;
+                            const int c = c0 + cl;
+                            if (MODE == kMatvec) {
+                                p.y[(int64_t)c * p.O + o] = v0[n][i];
+                            } else if (MODE == kGateUp) {
+                                ((uint16_t *)p.h)[(int64_t)c * p.O + o] =
+                                    (uint16_t)bf16_bits_rn(silu_mul(v0[n][i], v1[n][i]));
+                            } else if (MODE == kMoeGateUp) {
+                                ((uint16_t *)p.h)[(int64_t)(row0 + c) * p.O + o] =
+                                    (uint16_t)bf16_bits_rn(silu_mul(v0[n][i], v1[n][i]));
+                            } else {
+                                const int r = row0 + c;
+                                atomicAdd(p.y + (int64_t)p.row_tok[r] * p.O + o, p.wts[p.row_slot[r]] * v0[n][i]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+    // copies still in flight (only after an abort) must land before the CTA leaves
+    if (warp == kStConsumerWarps && lane == 0) {
+        const uint32_t first = issued > (uint32_t)NS ? issued - NS : 0;
+        for (uint32_t j = first; j < issued; ++j) {
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait(full_bar(j % NS), (j / NS) & 1) && global_ns() - t0 < 100000000ull) {
+            }
+        }
+    }
+    __syncthreads();
+}
+
+}  // namespace gq4
