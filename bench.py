@@ -184,7 +184,10 @@ def stage_work(cfg, sp):
 
 
 def stage_kernels(cfg, sp):
-    few = "gq4_band_kernel" if min(cfg.T, 23 if sp["tc"] else cfg.T) >= 3 else "gq4_skinny_kernel"
+    if cfg.H % 256 == 0 and cfg.F % 256 == 0:
+        few = "gq4_stream_kernel"  # TMA-fed decode kernel (whole four-group stages)
+    else:
+        few = "gq4_band_kernel" if min(cfg.T, 23 if sp["tc"] else cfg.T) >= 3 else "gq4_skinny_kernel"
     n = cfg.T * cfg.K
     route = "gq4_route_rowmap_small_kernel" if n <= 1024 else \
         "gq4_route_kernel + gq4_rowmap_{count,scan,fill}_kernel"
@@ -279,23 +282,30 @@ def main():
     cnt = ws.routing()["cnt"].cpu().numpy()[:cfg.E]
     split = split_experts(cfg, cnt)
 
-    # ---- device-timed steps (L2 flushed between steps, outside the events)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NEV)] for _ in range(args.steps)]
-    for row in evs:  # torch creates the CUDA event lazily, at its first record
-        for e in row:
-            e.record(stream)
+    # ---- device-timed steps: one moe_expert_ffn call (with its stage events) captured in
+    # a CUDA graph and replayed, so the step's kernels run without host launch gaps; L2
+    # flushed between steps, outside the events
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(NEV)]
+    for e in ev:  # torch creates the CUDA event lazily, at its first record
+        e.record(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(ev)
+    for _ in range(args.warmup):
+        graph.replay()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    stage = np.zeros((args.steps, NEV - 1))
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
-            step(evs[i])
-        torch.cuda.synchronize()
+            graph.replay()
+            torch.cuda.synchronize()
+            stage[i] = [ev[j].elapsed_time(ev[j + 1]) for j in range(NEV - 1)]
     if world > 1:
         dist.barrier()
-    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(NEV - 1)]
-                      for i in range(args.steps)])
     step_ms = stage.sum(1)
     ms = float(step_ms.mean())
 
@@ -329,7 +339,9 @@ def main():
     work = stage_work(cfg, split)
     kern = stage_kernels(cfg, split)
     t_stage = {k: float(stage[:, i].mean()) for i, k in enumerate(STAGES)}
-    dom = max(STAGES[1:], key=lambda k: t_stage[k])
+    busy = [k for k in STAGES[1:] if work[k][0] > 0 and (k.endswith("small") and split["n_small"] or
+                                                         k.endswith("large") and split["n_large"])]
+    dom = max(busy or STAGES[1:], key=lambda k: t_stage[k])
     dbytes, dflops = work[dom]
     if dflops > 0:
         roof = {"bound": "tensor", "achieved": dflops / (t_stage[dom] * 1e-3) / 1e12, "peak": bf16,
@@ -361,6 +373,7 @@ def main():
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "F": cfg.F, "K": cfg.K,
                        "gs": 64, "distinct_experts": n_active, "experts_tensor_core": split["n_large"],
                        "parallelism": f"replicas x{world}",
+                       "launch": "value: CUDA-graph replay of one moe_expert_ffn call; e2e: direct calls",
                        "l2": f"{L2_FLUSH_BYTES >> 20} MiB flush between steps; touched weights "
                              f"{n_active * per_expert / 1e9:.2f} GB/step"},
             "hbm_gbs_step": step_bytes / (ms * 1e-3) / 1e9,

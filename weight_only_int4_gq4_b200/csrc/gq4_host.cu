@@ -671,11 +671,14 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
 
     cudaStream_t s = S(stream);
     auto mark = [&](int i) {
-        if (stage_events && stage_events[i]) cudaEventRecord((cudaEvent_t)stage_events[i], s);
+        // external: inside a stream capture the record becomes a timestamped graph node
+        if (stage_events && stage_events[i])
+            cudaEventRecordWithFlags((cudaEvent_t)stage_events[i], s, cudaEventRecordExternal);
     };
     const int n = (int)(T * K);
     mark(0);
-    if (cudaMemsetAsync(at<int32_t>(ws, L.status), 0, 16, s) != cudaSuccess) return GQ4_ERR_CUDA;
+    // the one-block decode router clears the status word itself; the chunked path needs a memset
+    if (n > kChunk && cudaMemsetAsync(at<int32_t>(ws, L.status), 0, 16, s) != cudaSuccess) return GQ4_ERR_CUDA;
     // an expert can reach kLargeMin rows only if T does; the tensor-core kernels tile the
     // down rows by 128 and load scales four groups at a time
     const bool tc = T >= kLargeMin && H % 128 == 0 && F % 64 == 0 && Wg->ng % 4 == 0 && Wd->ng % 4 == 0 &&
@@ -739,8 +742,10 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     if (tc) {
         const int max_large = std::max(1, std::min<int>(E, (int)(T * K / kLargeMin)));
         const int chunks = (int)(H / 8);
-        gq4_gather_rows_kernel<<<sm_count() * 8, 256, 0, s>>>((const uint4 *)x, at<int32_t>(ws, L.row_tok),
-                                                             n, chunks, at<uint4>(ws, L.xg));
+        gq4_gather_rows_kernel<<<sm_count() * 4, 256, 0, s>>>((const uint4 *)x, at<int32_t>(ws, L.row_tok),
+                                                             at<int32_t>(ws, L.offs), at<int32_t>(ws, L.cnt),
+                                                             lists.n_large, lists.large, chunks,
+                                                             at<uint4>(ws, L.xg));
         if (cudaGetLastError() != cudaSuccess) return GQ4_ERR_CUDA;
         const uint64_t rows_gu = (uint64_t)(Wg->n_experts - 1) * (Wg->expert_stride_w / (H / 2)) + F;
         const uint64_t rows_d = (uint64_t)(Wd->n_experts - 1) * (Wd->expert_stride_w / (F / 2)) + H;

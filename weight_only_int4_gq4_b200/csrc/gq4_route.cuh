@@ -235,7 +235,8 @@ __global__ void __launch_bounds__(1024) gq4_rowmap_fill_kernel(const int32_t *id
 }
 
 // Decode path: router and the whole row map in one block of 1024 threads (T*K <= 1024).
-// Dynamic shared memory: (32 + 1) * E ints.
+// The block first clears the four-word status block (the layer's first kernel: nothing
+// else has written it yet).  Dynamic shared memory: (32 + 1) * E ints.
 template <int EPL>
 __global__ void __launch_bounds__(1024) gq4_route_rowmap_small_kernel(
     const float *logits, int T, int E, int K, int32_t *idx, float *wts, int32_t *status,
@@ -246,6 +247,8 @@ __global__ void __launch_bounds__(1024) gq4_route_rowmap_small_kernel(
     int32_t *wcnt = sm_dyn + E;    // [32][E]
     __shared__ int sh[32];
     const int warp = threadIdx.x >> 5;
+    if (threadIdx.x < 4) status[threadIdx.x] = 0;
+    __syncthreads();
     for (int t = warp; t < T; t += 32)
         route_token_warp<EPL>(logits + (int64_t)t * E, E, K, idx + (int64_t)t * K,
                               wts + (int64_t)t * K, status);
@@ -277,14 +280,26 @@ __global__ void __launch_bounds__(1024) gq4_route_rowmap_small_kernel(
 }  // namespace gq4
 
 namespace gq4 {
-// Gather the activation rows of the row map into row-map order: xg[r] = x[row_tok[r]].
-__global__ void gq4_gather_rows_kernel(const uint4 *x, const int32_t *row_tok, int n_rows,
+// Gather the activation rows of the experts with many rows into row-map order:
+// xg[r] = x[row_tok[r]] for every row r of an expert in the `large` list (the tensor-core
+// kernels read only those rows).  One warp per (large expert, row) pair.
+__global__ void gq4_gather_rows_kernel(const uint4 *x, const int32_t *row_tok, const int32_t *offs,
+                                       const int32_t *cnt, const int32_t *n_large, const int32_t *large,
                                        int chunks_per_row, uint4 *xg) {
-    const int64_t total = (int64_t)n_rows * chunks_per_row;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / chunks_per_row, c = i - r * chunks_per_row;
-        xg[i] = x[(int64_t)row_tok[r] * chunks_per_row + c];
+    const int nl = *n_large;
+    const int lane = threadIdx.x & 31;
+    const int warps = (gridDim.x * blockDim.x) >> 5;
+    int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    for (int a = 0; a < nl; ++a) {
+        const int e = large[a];
+        const int r0 = offs[e], n = cnt[e];
+        for (; w < n; w += warps) {
+            const int r = r0 + w;
+            const uint4 *src = x + (int64_t)row_tok[r] * chunks_per_row;
+            uint4 *dst = xg + (int64_t)r * chunks_per_row;
+            for (int c = lane; c < chunks_per_row; c += 32) dst[c] = src[c];
+        }
+        w -= n;  // continue the warp's stride in the next expert's rows
     }
 }
 }  // namespace gq4
