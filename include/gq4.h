@@ -191,8 +191,10 @@ gq4_status gq4_rowmap(const int32_t *idx, int64_t T, int32_t K, int32_t E, int32
  *   experts with many rows (row gather + tensor-core kernel), [4] after down of the
  *   experts with few rows, [5] after down of the experts with many rows.  Where a stage
  *   launches nothing its two events are recorded back to back.  A caller times the
- *   stages with cudaEventElapsedTime.  The events are recorded as external events, so a
- *   call captured in a CUDA graph records them at every replay. */
+ *   stages with cudaEventElapsedTime.  Inside a stream capture the events are recorded
+ *   as external events, so a call captured in a CUDA graph records them at every replay.
+ *   An event that cannot be recorded makes the call return GQ4_ERR_CUDA after its
+ *   launches. */
 #define GQ4_MOE_STAGE_EVENTS 6
 #define GQ4_MOE_LARGE_MIN_ROWS 24
 size_t moe_expert_ffn_workspace_bytes(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F);

@@ -304,3 +304,30 @@ def test_moe_prefill_full_size():
     s.check(y, ws, tokens)
     del s
     torch.cuda.empty_cache()
+
+
+def test_moe_stage_events_direct_and_in_cuda_graph():
+    """Stage events work on a plain call and inside a captured CUDA graph; the graph's
+    replays reproduce the plain call's output."""
+    s = MoESet(_toy(12, 16, 4, 256, 256))
+    lg = torch.from_numpy(s.lg).cuda()
+    x = bf16_to_torch(s.x)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(gq4.MOE_STAGE_EVENTS)]
+    for e in ev:
+        e.record()
+    y_ref, ws = gq4.moe_expert_ffn(s.Wg, s.Wu, s.Wd, lg, x, s.cfg.K, stage_events=ev)
+    torch.cuda.synchronize()
+    t = [ev[i].elapsed_time(ev[i + 1]) for i in range(gq4.MOE_STAGE_EVENTS - 1)]
+    assert all(v >= 0 for v in t) and sum(t) > 0
+    y = torch.empty_like(y_ref)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gq4.moe_expert_ffn(s.Wg, s.Wu, s.Wd, lg, x, s.cfg.K, y=y, ws=ws, stage_events=ev)
+    for _ in range(2):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        t = [ev[i].elapsed_time(ev[i + 1]) for i in range(gq4.MOE_STAGE_EVENTS - 1)]
+        assert all(v >= 0 for v in t) and sum(t) > 0
+        assert torch.allclose(y, y_ref, rtol=1e-5, atol=1e-4)
+    del g

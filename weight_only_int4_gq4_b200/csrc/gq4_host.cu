@@ -670,10 +670,20 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     if (overlap(yr, wr)) return GQ4_ERR_ALIAS;
 
     cudaStream_t s = S(stream);
+    bool marks_ok = true;  // a failed event record is reported after the launches
     auto mark = [&](int i) {
-        // external: inside a stream capture the record becomes a timestamped graph node
-        if (stage_events && stage_events[i])
-            cudaEventRecordWithFlags((cudaEvent_t)stage_events[i], s, cudaEventRecordExternal);
+        if (!stage_events || !stage_events[i]) return;
+        // inside a stream capture the record must be external to become a timestamped
+        // graph node; outside a capture the flag is not accepted
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        cudaStreamIsCapturing(s, &cap);
+        const cudaError_t e = cap == cudaStreamCaptureStatusActive
+                                  ? cudaEventRecordWithFlags((cudaEvent_t)stage_events[i], s, cudaEventRecordExternal)
+                                  : cudaEventRecord((cudaEvent_t)stage_events[i], s);
+        if (e != cudaSuccess) {
+            marks_ok = false;
+            cudaGetLastError();  // do not let it be read as a failed launch
+        }
     };
     const int n = (int)(T * K);
     mark(0);
@@ -797,7 +807,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
         st = launch_tc<1>(tm_d, tm_d, tm_h, td, max_large * td.m_tiles, s);
     }
     mark(5);
-    return st;
+    return st != GQ4_OK ? st : (marks_ok ? GQ4_OK : GQ4_ERR_CUDA);
 }
 
 }  // extern "C"
