@@ -196,7 +196,7 @@ gq4_status gq4_rowmap(const int32_t *idx, int64_t T, int32_t K, int32_t E, int32
  *   An event that cannot be recorded makes the call return GQ4_ERR_CUDA after its
  *   launches. */
 #define GQ4_MOE_STAGE_EVENTS 6
-#define GQ4_MOE_LARGE_MIN_ROWS 24
+#define GQ4_MOE_LARGE_MIN_ROWS 33
 size_t moe_expert_ffn_workspace_bytes(int64_t T, int32_t E, int32_t K, int64_t H, int64_t F);
 gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_tensor *Wd,
                           const float *logits, const void *x, gq4_dtype xdt, int64_t T,

@@ -77,6 +77,14 @@ def lib() -> ctypes.CDLL:
         L.orc_moe_tokens.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, I64,
                                      P, I, I, P, P, I64, P, I64, P, P]
         L.orc_moe_tokens.restype = None
+        L.orc_detect_group_size.argtypes = [I64, I64, I64]
+        L.orc_detect_group_size.restype = I64
+        L.orc_quantize.argtypes = [P, I64, I64, I64, P, P]
+        L.orc_quantize.restype = None
+        L.orc_dequant_rows.argtypes = [P, P, I64, I64, I64, P, I64, P, I, P]
+        L.orc_dequant_rows.restype = None
+        L.orc_matvec_rows.argtypes = [P, P, I64, I64, I64, P, I64, P, I, I64, P, P]
+        L.orc_matvec_rows.restype = None
     return _lib
 
 
@@ -243,4 +251,51 @@ def moe_tokens(pg, sg, pu, su, pd, sd, H, F, x, idx, wts, tokens, gs: int = 64,
     lib().orc_moe_tokens(_p(pg), _p(sg), _p(pu), _p(su), _p(pd), _p(sd), wgu, sgu, wd, sdd,
                          H, F, gs, _p(x), xdt, hdt, _p(idx), _p(wts), K, _p(tokens), n,
                          _p(y), _p(b))
+    return y, b
+
+
+# ------------------------------------------------------------------ NEXT rows
+def detect_group_size(O: int, I: int, scale_bytes: int) -> int:
+    """The one candidate group size matching the scale array's size; 0 none, -1 several."""
+    return lib().orc_detect_group_size(O, I, scale_bytes)
+
+
+def quantize(w, gs: int = 64):
+    """w f32 [O][I] -> (q int8 [O][I], scales f32 [O][ceil(I/gs)])."""
+    w = _c(w, np.float32)
+    O, I = w.shape
+    q = np.empty((O, I), np.int8)
+    s = np.empty((O, ngroups(I, gs)), np.float32)
+    lib().orc_quantize(_p(w), O, I, gs, _p(q), _p(s))
+    return q, s
+
+
+def dequant_rows(packed, scales, I, idx, gs: int = 64, alpha=None, out=None):
+    """out [n][I] fp64: alpha_j * w(idx[j], :) (+ out when out is given)."""
+    packed = _c(packed, np.uint8)
+    scales = _c(scales, np.float32)
+    idx = _c(idx, np.int32)
+    n = idx.shape[0]
+    acc = out is not None
+    o = _c(out, np.float64).copy() if acc else np.empty((n, I), np.float64)
+    a = None if alpha is None else _c(alpha, np.float64)
+    lib().orc_dequant_rows(_p(packed), _p(scales), packed.shape[0], I, gs, _p(idx), n,
+                           None if a is None else _p(a), int(acc), _p(o))
+    return o
+
+
+def matvec_rows(packed, scales, idx, x, gs: int = 64):
+    """y [T][n] fp64 over the rows idx, and the Sigma|terms| bound."""
+    packed = _c(packed, np.uint8)
+    scales = _c(scales, np.float32)
+    idx = _c(idx, np.int32)
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None]
+    T, I = x.shape
+    n = idx.shape[0]
+    y = np.empty((T, n), np.float64)
+    b = np.empty((T, n), np.float64)
+    lib().orc_matvec_rows(_p(packed), _p(scales), packed.shape[0], I, gs, _p(idx), n, _p(x),
+                          _xdt(x), T, _p(y), _p(b))
     return y, b

@@ -351,3 +351,102 @@ void orc_moe_tokens(const uint8_t *pg, const float *sg, const uint8_t *pu, const
     free(hmax);
     free(l1);
 }
+
+/* ---------------------------------------------------------------------------------
+ * NEXT rows: group-size detection, quantisation, row dequantisation / gather and the
+ * matvec over selected rows.
+ * ------------------------------------------------------------------------------- */
+
+/* detect_group_size.  [PR298] "What was implemented (CPU)": detect_group_size() derives
+ * gs from the byte count of the scale array, trying {16,32,48,64,96,128,192,256}.
+ * Reading: a candidate matches when O*ceil(I/gs)*4 equals the byte count; the answer is
+ * the single matching candidate.  Returns the group size, 0 when none matches, -1 when
+ * more than one matches (their groups differ, so the size cannot decide). */
+int64_t orc_detect_group_size(int64_t O, int64_t I, int64_t scale_bytes)
+{
+    static const int64_t cand[8] = {16, 32, 48, 64, 96, 128, 192, 256};
+    int64_t found = 0;
+    for (int c = 0; c < 8; c++) {
+        if (orc_scale_bytes(O, I, cand[c]) != scale_bytes) continue;
+        if (found) return -1;
+        found = cand[c];
+    }
+    return found;
+}
+
+/* Quantisation of float weights into the grouped format (the converter step before
+ * packing: [PR298] maintainer's "data request", "convert_fp8_to_int4.py --group-size 64").
+ * The pages name the group-size option, not the rounding.  Reading: a symmetric
+ * absmax scale per group, s = max|w| / 7, so the largest magnitude maps to +-7;
+ * q = round-half-to-even(w / s), clamped to [-8, 7]; an all-zero group gets s = 0 and
+ * q = 0.  The code is an integer decided by floating point, so the decision is taken in
+ * f32 (single-precision division and rounding), the precision the GPU kernel uses.
+ * Weights must be finite.  Output: q int8 [O][I] and scales f32 [O][ceil(I/gs)]; the
+ * last group may be partial; gs >= I gives one group per row (the per-row fmt=2 case). */
+void orc_quantize(const float *w, int64_t O, int64_t I, int64_t gs, int8_t *q, float *scales)
+{
+    int64_t ng = orc_ngroups(I, gs);
+    for (int64_t o = 0; o < O; o++)
+        for (int64_t g = 0; g < ng; g++) {
+            int64_t k0 = g * gs, k1 = k0 + gs < I ? k0 + gs : I;
+            float amax = 0.0f;
+            for (int64_t k = k0; k < k1; k++) {
+                float a = fabsf(w[o * I + k]);
+                if (a > amax) amax = a;
+            }
+            volatile float s = amax / 7.0f;  /* f32 division, no contraction */
+            scales[o * ng + g] = s;
+            for (int64_t k = k0; k < k1; k++) {
+                int v = 0;
+                if (s > 0.0f) {
+                    volatile float r = w[o * I + k] / s;
+                    float rq = rintf(r);  /* round half to even (default rounding mode) */
+                    if (rq > 7.0f) rq = 7.0f;
+                    if (rq < -8.0f) rq = -8.0f;
+                    v = (int)rq;
+                }
+                q[o * I + k] = (int8_t)v;
+            }
+        }
+}
+
+/* Row dequantisation / gather ([PR298] "embed_row, qt_addrow, qt_matvec_rows: fmt=4
+ * branches"): out[j][k] = (accumulate ? out[j][k] : 0) + alpha_j * w(idx[j], k), fp64,
+ * alpha_j = 1 when alpha is NULL.  embed_row is accumulate = 0 (a gather of dequantised
+ * rows), qt_addrow is accumulate = 1. */
+void orc_dequant_rows(const uint8_t *packed, const float *scales, int64_t O, int64_t I,
+                      int64_t gs, const int32_t *idx, int64_t n, const double *alpha,
+                      int accumulate, double *out)
+{
+    for (int64_t j = 0; j < n; j++) {
+        double a = alpha ? alpha[j] : 1.0;
+        for (int64_t k = 0; k < I; k++) {
+            double v = a * orc_weight(packed, scales, O, I, gs, idx[j], k);
+            out[j * I + k] = accumulate ? out[j * I + k] + v : v;
+        }
+    }
+}
+
+/* Matvec over selected rows (qt_matvec_rows): y[t][j] = sum_k w(idx[j], k) * x[t][k],
+ * natural k order, fp64; bound[t][j] = ||w_row||_1 * max_k |x[t][k]| as for orc_matvec. */
+void orc_matvec_rows(const uint8_t *packed, const float *scales, int64_t O, int64_t I,
+                     int64_t gs, const int32_t *idx, int64_t n, const void *x, int xdt,
+                     int64_t T, double *y, double *bound)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < n; j++) {
+        int64_t o = idx[j];
+        double l1 = 0.0;
+        for (int64_t k = 0; k < I; k++) l1 += fabs(orc_weight(packed, scales, O, I, gs, o, k));
+        for (int64_t t = 0; t < T; t++) {
+            double acc = 0.0, xmax = 0.0;
+            for (int64_t k = 0; k < I; k++) {
+                double xv = orc_x(x, xdt, t * I + k);
+                acc += orc_weight(packed, scales, O, I, gs, o, k) * xv;
+                if (fabs(xv) > xmax) xmax = fabs(xv);
+            }
+            y[t * n + j] = acc;
+            if (bound) bound[t * n + j] = l1 * xmax;
+        }
+    }
+}

@@ -243,7 +243,7 @@ def _toy(T, E, K, H=128, F=128, seed=3, **kw):
 @pytest.mark.parametrize("T,E,K,H,F", [(5, 4, 2, 128, 128), (1, 1, 1, 64, 64), (3, 8, 8, 192, 256),
                                        (17, 16, 4, 256, 128), (40, 32, 8, 128, 192),
                                        (300, 16, 4, 128, 64),
-                                       # tensor-core path (experts with >= 24 rows), mixed with
+                                       # tensor-core path (experts with >= 33 rows), mixed with
                                        # the decode path, multi-pass experts (> 192 rows)
                                        (64, 4, 2, 256, 128), (40, 8, 4, 384, 192), (300, 2, 1, 128, 64),
                                        (500, 2, 2, 128, 128), (48, 4, 2, 192, 128), (130, 6, 3, 512, 256),

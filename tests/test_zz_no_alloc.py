@@ -39,10 +39,10 @@ def _noalloc(W, lg, x, K, y, status):
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_two_calls():
     torch.cuda.set_device(0)
-    # first call: few rows per expert (decode kernels); second call: experts with at least
-    # 24 rows (row gather + tensor-core kernels, which use more of the array)
+    # first call: few rows per expert (decode kernels); second call: experts with more
+    # than 32 rows (row gather + tensor-core kernels, which use more of the array)
     cases = [synth.MoEConfig("noalloc_t6_e8_k2", T=6, H=256, E=8, F=128, K=2, seed=41),
-             synth.MoEConfig("noalloc_t40_e4_k2", T=40, H=256, E=4, F=128, K=2, seed=42)]
+             synth.MoEConfig("noalloc_t80_e4_k2", T=80, H=256, E=4, F=128, K=2, seed=42)]
     for cfg in cases:
         st = _stacked(cfg)
         W = {n: gq4.upload(*st[n]) for n in st}

@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgq4.so")
 ABI_VERSION = 2
 MOE_STAGE_EVENTS = 6
-MOE_LARGE_MIN_ROWS = 24  # GQ4_MOE_LARGE_MIN_ROWS
+MOE_LARGE_MIN_ROWS = 33  # GQ4_MOE_LARGE_MIN_ROWS
 NOALLOC_SCRATCH_BYTES = 16 << 20  # GQ4_NOALLOC_SCRATCH_BYTES
 
 OK, ERR_NULL, ERR_ALIGN, ERR_SHAPE, ERR_UNSUPPORTED, ERR_ALIAS, ERR_WORKSPACE, ERR_CUDA, \
