@@ -26,8 +26,10 @@
  *     (pxq_llama.cpp release notes 2026-09-02, "Host-overhead cuts": the router aliasing
  *     barrier; "Correctness fixes": a fused path that did not check 16-byte base
  *     alignment faulted instead of declining -- here the call declines).
- *   - The GPU kernels take gs = 64 and in % 64 == 0; other group sizes and partial last
- *     groups return GQ4_ERR_UNSUPPORTED (the host packer accepts any shape).
+ *   - The fast kernels take gs = 64 and in % 64 == 0; the matvec, gate+up, row and
+ *     quantisation calls also take any gs that is a multiple of 8 with in % 8 == 0
+ *     (partial last groups included) on generic kernels; moe_expert_ffn needs gs = 64.
+ *     Other shapes return GQ4_ERR_UNSUPPORTED (the host packer accepts any shape).
  *   - No call keeps global mutable state, reads environment variables or throws.
  */
 #ifndef GQ4_H
@@ -213,6 +215,56 @@ gq4_status moe_expert_ffn_routing(void *ws, size_t ws_bytes, int64_t T, int32_t 
 gq4_status moe_expert_ffn_status(const void *ws, size_t ws_bytes, int64_t T, int32_t E,
                                  int32_t K, int64_t H, int64_t F, gq4_stream_t stream,
                                  int32_t *status);
+
+/* ---------------------------------------------------------------- general group sizes,
+ * quantisation and row operations (any gs that is a multiple of 8; in % 8 == 0)
+ *
+ * gq4_matvec and gq4_gate_up_silu above take these shapes too: a tensor with gs != 64
+ * or a partial last group runs on a generic CUDA-core kernel (one warp per row, the
+ * scale applied once per group), colibri PR #298 "What was implemented (CPU)":
+ * matmul_i4_grouped "handles arbitrary gs (multiple of 16)".  Only moe_expert_ffn still
+ * requires gs = 64 and in % 64 == 0.
+ *
+ * gq4_detect_group_size: host only.  The group size of a matrix from the byte count of
+ * its scale array (PR #298, same section: detect_group_size() tries
+ * {16,32,48,64,96,128,192,256}): *gs_out = the one candidate with
+ * out*ceil(in/gs)*4 == scale_bytes.  GQ4_ERR_SHAPE when none matches,
+ * GQ4_ERR_UNSUPPORTED when two or more match (their groups differ; the size alone
+ * cannot decide). */
+gq4_status gq4_detect_group_size(int64_t out, int64_t in, size_t scale_bytes, int32_t *gs_out);
+
+/* gq4_quantize: float weights -> grouped int4 in the device layout, on the GPU (the
+ * converter step, PR #298 maintainer's "data request": convert_fp8_to_int4.py
+ * --group-size 64).  Per group of gs consecutive inputs of a row (the last group of a
+ * row may be partial; gs >= in gives one scale per row, the fmt=2 case):
+ *   s = max|w| / 7 (f32 division), q = round-half-to-even(w / s) in f32, clamped to
+ *   [-8, 7]; an all-zero group gets s = 0 and q = 0.
+ * The pages name the group size, not the rounding: this absmax rule is the reading.
+ *   w: device f32 [out][in], 16-byte aligned, finite; d_w: device, >= out*in/2 bytes;
+ *   d_s: device f32 [out][ceil(in/gs)]; *desc filled as gq4_tensor_init does.
+ *   gs % 8 == 0 and in % 8 == 0 (GQ4_ERR_UNSUPPORTED otherwise). */
+gq4_status gq4_quantize(const float *w, int64_t out, int64_t in, int32_t gs, void *d_w,
+                        size_t d_w_bytes, float *d_s, size_t d_s_bytes, gq4_stream_t stream,
+                        gq4_tensor *desc);
+
+/* gq4_dequant_rows: row dequantisation / gather (PR #298: embed_row, qt_addrow and
+ * qt_matvec_rows needed the fmt=4 per-group-scale branch).
+ *   out[j][k] = (accumulate ? out[j][k] : 0) + alpha[j] * w[idx[j]][k], k < in,
+ * alpha = NULL meaning 1.  embed_row is accumulate = 0, qt_addrow accumulate = 1.
+ *   idx: device int32 [n]; alpha: NULL or device f32 [n]; out: device [n][in] of odt
+ *   (GQ4_F32, or GQ4_BF16 rounded to nearest even, which takes no accumulate).
+ *   An index outside [0, W->out) is not read: that row of out becomes NaN. */
+gq4_status gq4_dequant_rows(const gq4_tensor *W, const int32_t *idx, int64_t n,
+                            const float *alpha, int32_t accumulate, void *out, gq4_dtype odt,
+                            gq4_stream_t stream);
+
+/* gq4_matvec_rows: matvec over selected rows (qt_matvec_rows):
+ *   y[t][j] = sum_k w[idx[j]][k] * x[t][k], fp32 accumulation.
+ *   idx: device int32 [n_sel]; x: device [n_tok][W->in] of xdt; y: device f32
+ *   [n_tok][n_sel].  An index outside [0, W->out) gives NaN in its column of y. */
+gq4_status gq4_matvec_rows(const gq4_tensor *W, const int32_t *idx, int64_t n_sel,
+                           const void *x, gq4_dtype xdt, int64_t n_tok, float *y,
+                           gq4_stream_t stream);
 
 /* moe_expert_ffn_noalloc: the same layer as moe_expert_ffn, for callers that cannot
  * allocate device memory -- a plug-in whose host program owns every device allocation

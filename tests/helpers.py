@@ -24,6 +24,20 @@ def torch_bf16_to_bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
+def device_words_to_host(dev: np.ndarray) -> np.ndarray:
+    """Undo the device nibble order (even-k nibbles in the low half-word, odd-k in the
+    high half-word of each 32-bit word) to get the pages' low-nibble-first bytes."""
+    w = dev.reshape(dev.shape[0], -1).view(np.uint32)
+    nib = np.stack([(w >> (4 * i)) & 15 for i in range(8)], -1)  # slots 0..7
+    k = np.empty_like(nib)
+    k[..., 0::2] = nib[..., 0:4]
+    k[..., 1::2] = nib[..., 4:8]
+    host = np.zeros_like(w)
+    for i in range(8):
+        host |= (k[..., i] << (4 * i)).astype(np.uint32)
+    return host.view(np.uint8).reshape(dev.shape)
+
+
 def check_close(y_gpu, y_orc, bound, what=""):
     y_gpu = np.asarray(y_gpu, np.float64)
     y_orc = np.asarray(y_orc, np.float64)

@@ -77,8 +77,8 @@ def test_matvec_argument_checks():
     assert _matvec(_desc(), x=0) == gq4.ERR_NULL
     assert _matvec(_desc(w=0x10008)) == gq4.ERR_ALIGN
     assert _matvec(_desc(), y=0x40004) == gq4.ERR_ALIGN
-    assert _matvec(_desc(gs=32)) == gq4.ERR_UNSUPPORTED          # gs != 64
-    assert _matvec(_desc(in_=100)) == gq4.ERR_UNSUPPORTED        # partial last group
+    assert _matvec(_desc(gs=12)) == gq4.ERR_UNSUPPORTED          # gs not a multiple of 8
+    assert _matvec(_desc(in_=100)) == gq4.ERR_UNSUPPORTED        # in not a multiple of 8
     bad = _desc()
     bad.ng = 3
     assert _matvec(bad) == gq4.ERR_SHAPE                          # ng inconsistent with in
@@ -137,8 +137,50 @@ def test_moe_argument_checks():
     assert call(y=0x710000) == gq4.ERR_ALIAS  # y over x
     assert call(ws=0x100000) == gq4.ERR_ALIAS  # workspace over gate weights
     assert call(logits=0) == gq4.ERR_NULL
+    assert call(g=_desc(out=F, in_=H, gs=32, w=0x100000, s=0x200000, E=E)) == gq4.ERR_UNSUPPORTED  # MoE: gs 64
     r = gq4.RoutingDesc()
     assert L.moe_expert_ffn_routing(0x800000, ws_bytes, T, E, K, H, F, ctypes.byref(r)) == gq4.OK
     ptrs = [r.idx, r.wts, r.cnt, r.offs, r.row_tok, r.row_slot, r.slot_row, r.n_active, r.active, r.status]
     assert all(p % 16 == 0 and 0x800000 <= p < 0x800000 + ws_bytes for p in ptrs)
     assert len(set(ptrs)) == len(ptrs)
+
+
+def test_detect_group_size_host():
+    L = gq4.lib()
+    gs = ctypes.c_int32(0)
+    assert L.gq4_detect_group_size(28672, 512, 917504, ctypes.byref(gs)) == gq4.OK and gs.value == 64
+    assert L.gq4_detect_group_size(2048, 6144, 2048 * 48 * 4, ctypes.byref(gs)) == gq4.OK and gs.value == 128
+    assert L.gq4_detect_group_size(100, 4096, 123, ctypes.byref(gs)) == gq4.ERR_SHAPE
+    assert L.gq4_detect_group_size(100, 16, 400, ctypes.byref(gs)) == gq4.ERR_UNSUPPORTED
+    assert L.gq4_detect_group_size(100, 16, 400, None) == gq4.ERR_NULL
+    assert gq4.detect_group_size(6144, 2048, 6144 * 32 * 4) == 64
+
+
+def test_quantize_and_row_ops_argument_checks():
+    """Every rejected call returns before anything is launched (fake pointers)."""
+    L = gq4.lib()
+    d = gq4.TensorDesc()
+    q = lambda w=0x100000, O=64, I=128, gs=64, dw=0x200000, dwb=4096, ds=0x300000, dsb=512: \
+        L.gq4_quantize(w, O, I, gs, dw, dwb, ds, dsb, None, ctypes.byref(d))
+    assert q(w=0) == gq4.ERR_NULL
+    assert q(gs=12) == gq4.ERR_UNSUPPORTED
+    assert q(I=100) == gq4.ERR_UNSUPPORTED
+    assert q(dwb=4095) == gq4.ERR_SHAPE
+    assert q(w=0x100004) == gq4.ERR_ALIGN
+    assert q(dw=0x100000) == gq4.ERR_ALIAS
+    W = _desc()
+    dr = lambda idx=0x500000, n=3, alpha=None, acc=0, out=0x600000, odt=0, d=W: \
+        L.gq4_dequant_rows(ctypes.byref(d), idx, n, alpha, acc, out, odt, None)
+    assert dr(idx=0) == gq4.ERR_NULL
+    assert dr(n=0) == gq4.ERR_SHAPE
+    assert dr(odt=1, acc=1) == gq4.ERR_UNSUPPORTED
+    assert dr(out=0x600008) == gq4.ERR_ALIGN
+    assert dr(out=0x10000) == gq4.ERR_ALIAS
+    assert dr(d=_desc(gs=12)) == gq4.ERR_UNSUPPORTED
+    mr = lambda idx=0x500000, n=3, x=0x700000, xdt=1, T=1, y=0x800000: \
+        L.gq4_matvec_rows(ctypes.byref(W), idx, n, x, xdt, T, y, None)
+    assert mr(x=0) == gq4.ERR_NULL
+    assert mr(T=0) == gq4.ERR_SHAPE
+    assert mr(xdt=5) == gq4.ERR_UNSUPPORTED
+    assert mr(y=0x700000) == gq4.ERR_ALIAS
+    assert mr(idx=0x500002) == gq4.ERR_ALIGN

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle
-from tests.helpers import (bf16_to_torch, check_bf16_close, check_close, h_bound,
+from tests.helpers import (bf16_to_torch, check_bf16_close, check_close, device_words_to_host, h_bound,
                            torch_bf16_to_bits)
 from weight_only_int4_gq4_b200 import synth
 
@@ -15,20 +15,6 @@ pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     from weight_only_int4_gq4_b200 import gq4
-
-
-def device_words_to_host(dev: np.ndarray) -> np.ndarray:
-    """Undo the device nibble order (even-k nibbles in the low half-word, odd-k in the
-    high half-word of each 32-bit word) to get the pages' low-nibble-first bytes."""
-    w = dev.reshape(dev.shape[0], -1).view(np.uint32)
-    nib = np.stack([(w >> (4 * i)) & 15 for i in range(8)], -1)  # slots 0..7
-    k = np.empty_like(nib)
-    k[..., 0::2] = nib[..., 0:4]
-    k[..., 1::2] = nib[..., 4:8]
-    host = np.zeros_like(w)
-    for i in range(8):
-        host |= (k[..., i] << (4 * i)).astype(np.uint32)
-    return host.view(np.uint8).reshape(dev.shape)
 
 
 def _x_torch(x):

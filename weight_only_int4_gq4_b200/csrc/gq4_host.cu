@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "gq4.h"
+#include "gq4_aux.cuh"
 #include "gq4_common.cuh"
 #include "gq4_route.cuh"
 #include "gq4_skinny.cuh"
@@ -43,6 +44,18 @@ gq4_status check_tensor(const gq4_tensor *t, int n_experts_min) {
             return GQ4_ERR_SHAPE;
         if (t->expert_stride_w % 16 || t->expert_stride_s % 4) return GQ4_ERR_ALIGN;
     }
+    return GQ4_OK;
+}
+
+// Checks of one tensor descriptor for the generic kernels: any group size that is a
+// multiple of 8 (a device word of 8 weights lies in one group), in % 8 == 0.
+gq4_status check_tensor_generic(const gq4_tensor *t, int n_experts_min) {
+    if (!t || !t->w || !t->s) return GQ4_ERR_NULL;
+    if (t->out < 1 || t->in < 1 || t->n_experts < n_experts_min) return GQ4_ERR_SHAPE;
+    if (t->gs <= 0 || t->ng != (t->in + t->gs - 1) / t->gs) return GQ4_ERR_SHAPE;
+    if (t->gs % 8 != 0 || t->in % 8 != 0) return GQ4_ERR_UNSUPPORTED;
+    if (t->out > (int64_t)1 << 30 || t->in > (int64_t)1 << 20) return GQ4_ERR_SHAPE;
+    if (!aligned16(t->w) || !aligned16(t->s)) return GQ4_ERR_ALIGN;
     return GQ4_OK;
 }
 
@@ -404,6 +417,29 @@ gq4_status launch_tc(const CUtensorMap &w0, const CUtensorMap &w1, const CUtenso
 
 }  // namespace
 
+// ---- generic kernels (gq4_aux.cuh) ----------------------------------------------------
+// Matvec / gate+up over all rows or selected rows, any group size that is a multiple of 8.
+template <int MODE>
+gq4_status launch_generic(const gq4_tensor *W0, const gq4_tensor *W1, int64_t n_rows, const int32_t *rows,
+                          const void *x, gq4_dtype xdt, int64_t n_tok, void *out, cudaStream_t st) {
+    const size_t xbytes = (size_t)n_tok * W0->in * 4;
+    const int stage = xbytes <= 96 * 1024 ? 1 : 0;
+    const size_t smem = stage ? xbytes : 0;
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((n_rows + 7) / 8, (int64_t)sm_count() * 8));
+#define GEN_LAUNCH(XDT)                                                                                    \
+    {                                                                                                      \
+        auto kern = gq4_generic_kernel<MODE, XDT>;                                                         \
+        if (allow_smem(kern, smem) != cudaSuccess) return GQ4_ERR_CUDA;                                    \
+        kern<<<blocks, 256, smem, st>>>((const uint32_t *)W0->w, W0->s,                                    \
+                                        (const uint32_t *)(W1 ? W1->w : W0->w), W1 ? W1->s : W0->s,        \
+                                        W0->out, n_rows, rows, W0->in, W0->gs, W0->ng, x, (int)n_tok,      \
+                                        stage, out);                                                       \
+    }
+    if (xdt == GQ4_BF16) GEN_LAUNCH(1) else GEN_LAUNCH(0)
+#undef GEN_LAUNCH
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
 // =====================================================================================
 extern "C" {
 
@@ -502,7 +538,7 @@ gq4_status gq4_upload(const uint8_t *packed_host, const float *scales_host, int6
 
 gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t n_tok,
                       float *y, gq4_stream_t stream) {
-    gq4_status st = check_tensor(W, 1);
+    gq4_status st = check_tensor_generic(W, 1);
     if (st != GQ4_OK) return st;
     if (!x || !y) return GQ4_ERR_NULL;
     if (xdt != GQ4_F32 && xdt != GQ4_BF16) return GQ4_ERR_UNSUPPORTED;
@@ -513,6 +549,8 @@ gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t
     if (overlap(yr, rng(x, xb)) || overlap(yr, rng(W->w, tensor_w_bytes(W))) ||
         overlap(yr, rng(W->s, tensor_s_bytes(W))))
         return GQ4_ERR_ALIAS;
+    if (check_tensor(W, 1) != GQ4_OK)  // another group size or a partial last group
+        return launch_generic<0>(W, nullptr, W->out, nullptr, x, xdt, n_tok, y, S(stream));
     SkinnyParams p{};
     p.w0 = W->w; p.s0 = W->s;
     p.O = (int)W->out; p.I = (int)W->in; p.ng = W->ng;
@@ -529,11 +567,11 @@ gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t
 
 gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const void *x,
                             gq4_dtype xdt, int64_t n_tok, void *h, gq4_stream_t stream) {
-    gq4_status st = check_tensor(Wg, 1);
+    gq4_status st = check_tensor_generic(Wg, 1);
     if (st != GQ4_OK) return st;
-    st = check_tensor(Wu, 1);
+    st = check_tensor_generic(Wu, 1);
     if (st != GQ4_OK) return st;
-    if (Wg->out != Wu->out || Wg->in != Wu->in) return GQ4_ERR_SHAPE;
+    if (Wg->out != Wu->out || Wg->in != Wu->in || Wg->gs != Wu->gs) return GQ4_ERR_SHAPE;
     if (!x || !h) return GQ4_ERR_NULL;
     if (xdt != GQ4_F32 && xdt != GQ4_BF16) return GQ4_ERR_UNSUPPORTED;
     if (n_tok < 1 || n_tok > (1 << 20)) return GQ4_ERR_SHAPE;
@@ -544,6 +582,8 @@ gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const vo
         overlap(hr, rng(Wg->w, tensor_w_bytes(Wg))) || overlap(hr, rng(Wg->s, tensor_s_bytes(Wg))) ||
         overlap(hr, rng(Wu->w, tensor_w_bytes(Wu))) || overlap(hr, rng(Wu->s, tensor_s_bytes(Wu))))
         return GQ4_ERR_ALIAS;
+    if (check_tensor(Wg, 1) != GQ4_OK || check_tensor(Wu, 1) != GQ4_OK)  // general group size
+        return launch_generic<1>(Wg, Wu, Wg->out, nullptr, x, xdt, n_tok, h, S(stream));
     SkinnyParams p{};
     p.w0 = Wg->w; p.s0 = Wg->s; p.w1 = Wu->w; p.s1 = Wu->s;
     p.O = (int)Wg->out; p.I = (int)Wg->in; p.ng = Wg->ng;
@@ -868,4 +908,92 @@ extern "C" gq4_status moe_expert_ffn_noalloc(const gq4_tensor *Wg, const gq4_ten
         cudaSuccess)
         return GQ4_ERR_CUDA;
     return GQ4_OK;
+}
+
+// ---- group-size detection, quantisation, row dequantisation, matvec over rows ----------
+extern "C" gq4_status gq4_detect_group_size(int64_t out, int64_t in, size_t scale_bytes, int32_t *gs_out) {
+    if (!gs_out) return GQ4_ERR_NULL;
+    if (out < 1 || in < 1) return GQ4_ERR_SHAPE;
+    static const int32_t cand[8] = {16, 32, 48, 64, 96, 128, 192, 256};
+    int32_t found = 0;
+    for (int c = 0; c < 8; ++c) {
+        const int64_t ng = (in + cand[c] - 1) / cand[c];
+        if ((size_t)(out * ng * 4) != scale_bytes) continue;
+        if (found) return GQ4_ERR_UNSUPPORTED;  // two candidates give the same size
+        found = cand[c];
+    }
+    if (!found) return GQ4_ERR_SHAPE;
+    *gs_out = found;
+    return GQ4_OK;
+}
+
+extern "C" gq4_status gq4_quantize(const float *w, int64_t out, int64_t in, int32_t gs, void *d_w,
+                                   size_t d_w_bytes, float *d_s, size_t d_s_bytes, gq4_stream_t stream,
+                                   gq4_tensor *desc) {
+    if (!w || !d_w || !d_s || !desc) return GQ4_ERR_NULL;
+    if (out < 1 || in < 1 || gs < 1 || out > ((int64_t)1 << 30) || in > ((int64_t)1 << 20)) return GQ4_ERR_SHAPE;
+    if (in % 8 || gs % 8) return GQ4_ERR_UNSUPPORTED;
+    size_t wb = 0, sb = 0;
+    gq4_status st = gq4_device_bytes(out, in, gs, 1, &wb, &sb);
+    if (st != GQ4_OK) return st;
+    if (d_w_bytes < wb || d_s_bytes < sb) return GQ4_ERR_SHAPE;
+    if (!aligned16(w) || !aligned16(d_w) || !aligned16(d_s)) return GQ4_ERR_ALIGN;
+    const Range wr = rng(w, (size_t)out * in * 4), dwr = rng(d_w, wb), dsr = rng(d_s, sb);
+    if (overlap(wr, dwr) || overlap(wr, dsr) || overlap(dwr, dsr)) return GQ4_ERR_ALIAS;
+    const int ng = (int)((in + gs - 1) / gs);
+    const int words = (int)std::min<int64_t>(gs / 8, 32);
+    const int64_t groups = out * ng;
+    const cudaStream_t s = S(stream);
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((groups * 32 / std::max(words, 1) + 255) / 256,
+                                                                   (int64_t)sm_count() * 16));
+#define QLAUNCH(SEG) gq4_quantize_kernel<SEG><<<blocks, 256, 0, s>>>(w, out, in, gs, ng, (uint32_t *)d_w, d_s)
+    if (words <= 1) QLAUNCH(1);
+    else if (words <= 2) QLAUNCH(2);
+    else if (words <= 4) QLAUNCH(4);
+    else if (words <= 8) QLAUNCH(8);
+    else if (words <= 16) QLAUNCH(16);
+    else QLAUNCH(32);
+#undef QLAUNCH
+    if (cudaGetLastError() != cudaSuccess) return GQ4_ERR_CUDA;
+    return gq4_tensor_init(d_w, d_s, out, in, gs, 1, desc);
+}
+
+extern "C" gq4_status gq4_dequant_rows(const gq4_tensor *W, const int32_t *idx, int64_t n, const float *alpha,
+                                       int32_t accumulate, void *out, gq4_dtype odt, gq4_stream_t stream) {
+    gq4_status st = check_tensor_generic(W, 1);
+    if (st != GQ4_OK) return st;
+    if (!idx || !out) return GQ4_ERR_NULL;
+    if (n < 1 || n > ((int64_t)1 << 30)) return GQ4_ERR_SHAPE;
+    if (odt != GQ4_F32 && odt != GQ4_BF16) return GQ4_ERR_UNSUPPORTED;
+    if (odt == GQ4_BF16 && accumulate) return GQ4_ERR_UNSUPPORTED;
+    if (!aligned16(out) || !aligned16(idx) || (alpha && !aligned16(alpha))) return GQ4_ERR_ALIGN;
+    const Range orr = rng(out, (size_t)n * W->in * (odt == GQ4_F32 ? 4 : 2));
+    if (overlap(orr, rng(idx, (size_t)n * 4)) || overlap(orr, rng(W->w, tensor_w_bytes(W))) ||
+        overlap(orr, rng(W->s, tensor_s_bytes(W))) || (alpha && overlap(orr, rng(alpha, (size_t)n * 4))))
+        return GQ4_ERR_ALIAS;
+    const cudaStream_t s = S(stream);
+    const int64_t total = n * (W->in / 8);
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 16));
+    if (odt == GQ4_F32)
+        gq4_dequant_rows_kernel<0><<<blocks, 256, 0, s>>>((const uint32_t *)W->w, W->s, W->out, W->in, W->gs, W->ng,
+                                                          idx, n, alpha, accumulate, out);
+    else
+        gq4_dequant_rows_kernel<1><<<blocks, 256, 0, s>>>((const uint32_t *)W->w, W->s, W->out, W->in, W->gs, W->ng,
+                                                          idx, n, alpha, 0, out);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
+extern "C" gq4_status gq4_matvec_rows(const gq4_tensor *W, const int32_t *idx, int64_t n_sel, const void *x,
+                                      gq4_dtype xdt, int64_t n_tok, float *y, gq4_stream_t stream) {
+    gq4_status st = check_tensor_generic(W, 1);
+    if (st != GQ4_OK) return st;
+    if (!idx || !x || !y) return GQ4_ERR_NULL;
+    if (xdt != GQ4_F32 && xdt != GQ4_BF16) return GQ4_ERR_UNSUPPORTED;
+    if (n_sel < 1 || n_sel > ((int64_t)1 << 30) || n_tok < 1 || n_tok > (1 << 20)) return GQ4_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(idx)) return GQ4_ERR_ALIGN;
+    const Range yr = rng(y, (size_t)n_tok * n_sel * 4);
+    if (overlap(yr, rng(x, (size_t)n_tok * W->in * (xdt == GQ4_F32 ? 4 : 2))) || overlap(yr, rng(idx, (size_t)n_sel * 4)) ||
+        overlap(yr, rng(W->w, tensor_w_bytes(W))) || overlap(yr, rng(W->s, tensor_s_bytes(W))))
+        return GQ4_ERR_ALIAS;
+    return launch_generic<0>(W, nullptr, n_sel, idx, x, xdt, n_tok, y, S(stream));
 }

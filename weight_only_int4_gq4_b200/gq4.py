@@ -68,6 +68,10 @@ _SIGS = {
                               ctypes.c_int),
     "moe_expert_ffn_noalloc": ([_TP, _TP, _TP, _P, _P, ctypes.c_int, _I64, _I32, _I32, _P, _P, _P],
                                ctypes.c_int),
+    "gq4_detect_group_size": ([_I64, _I64, _SZ, ctypes.POINTER(_I32)], ctypes.c_int),
+    "gq4_quantize": ([_P, _I64, _I64, _I32, _P, _SZ, _P, _SZ, _P, _TP], ctypes.c_int),
+    "gq4_dequant_rows": ([_TP, _P, _I64, _P, _I32, _P, ctypes.c_int, _P], ctypes.c_int),
+    "gq4_matvec_rows": ([_TP, _P, _I64, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -332,4 +336,54 @@ def moe_expert_ffn_noalloc(Wg: Tensor, Wu: Tensor, Wd: Tensor, logits: torch.Ten
     _check(_lib.moe_expert_ffn_noalloc(Wg.ref(), Wu.ref(), Wd.ref(), logits.data_ptr(), x.data_ptr(),
                                        _xdt(x), T, E, K, y.data_ptr(), _ptr(status_out), _stream(stream)),
            "moe_expert_ffn_noalloc")
+    return y
+
+
+# ------------------------------------------------------------------ general group sizes, rows
+def detect_group_size(out: int, in_: int, scale_bytes: int) -> int:
+    """Group size of a matrix from its scale array's byte count (raises if none or ambiguous)."""
+    gs = _I32()
+    _check(_lib.gq4_detect_group_size(out, in_, scale_bytes, ctypes.byref(gs)), "gq4_detect_group_size")
+    return gs.value
+
+
+def quantize(w: torch.Tensor, gs: int = 64, stream=None) -> Tensor:
+    """f32 device weights [O][I] -> grouped-int4 Tensor (absmax scales, round half to even)."""
+    if w.dtype != torch.float32 or w.dim() != 2:
+        raise TypeError("quantize: expected a 2-D float32 tensor")
+    _need_cuda(w)
+    O, I = w.shape
+    wb, sb = device_bytes(O, I, gs, 1)
+    d_w = torch.empty(wb, dtype=torch.uint8, device=w.device)
+    d_s = torch.empty(sb // 4, dtype=torch.float32, device=w.device)
+    desc = TensorDesc()
+    _check(_lib.gq4_quantize(w.data_ptr(), O, I, gs, d_w.data_ptr(), wb, d_s.data_ptr(), sb, _stream(stream),
+                             ctypes.byref(desc)), "gq4_quantize")
+    return Tensor(desc, d_w, d_s)
+
+
+def dequant_rows(W: Tensor, idx: torch.Tensor, alpha: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                 accumulate: bool = False, dtype=torch.float32, stream=None) -> torch.Tensor:
+    """out [n][I] = (accumulate ? out : 0) + alpha[j] * w[idx[j]] (rows dequantised)."""
+    n = idx.shape[0]
+    if out is None:
+        out = torch.empty(n, W.in_, dtype=dtype, device=idx.device)
+    _need_cuda(idx, out, alpha)
+    odt = _xdt(out)
+    _check(_lib.gq4_dequant_rows(W.ref(), idx.data_ptr(), n, _ptr(alpha), int(accumulate), out.data_ptr(), odt,
+                                 _stream(stream)), "gq4_dequant_rows")
+    return out
+
+
+def matvec_rows(W: Tensor, idx: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """y [T][n] f32 = x [T][I] times the selected rows of W."""
+    if x.dim() == 1:
+        x = x[None]
+    n = idx.shape[0]
+    if y is None:
+        y = torch.empty(x.shape[0], n, dtype=torch.float32, device=x.device)
+    _need_cuda(idx, x, y)
+    _check(_lib.gq4_matvec_rows(W.ref(), idx.data_ptr(), n, x.data_ptr(), _xdt(x), x.shape[0], y.data_ptr(),
+                                _stream(stream)), "gq4_matvec_rows")
     return y
