@@ -394,14 +394,15 @@ gq4_status launch_stream_nt(const StreamMats &m, const SkinnyParams &p, int mats
     }
 }
 
+// At most three n-tiles (24 columns) per pass: the four-tile variant needs more registers
+// than the 16 consumer warps have and spills; a matrix with more columns takes passes.
 template <int MODE>
 gq4_status launch_stream(const StreamMats &m, const SkinnyParams &p, int max_cols, int mats, int32_t *status,
                          cudaStream_t st) {
     const int c = std::min(max_cols, kStMaxCols);
     if (c <= 8) return launch_stream_nt<MODE, 1>(m, p, mats, status, st);
     if (c <= 16) return launch_stream_nt<MODE, 2>(m, p, mats, status, st);
-    if (c <= 24) return launch_stream_nt<MODE, 3>(m, p, mats, status, st);
-    return launch_stream_nt<MODE, 4>(m, p, mats, status, st);
+    return launch_stream_nt<MODE, 3>(m, p, mats, status, st);
 }
 
 template <int MODE>

@@ -23,51 +23,66 @@ constexpr int kChunk = 1024;        // slots per row-map chunk (one per thread)
 constexpr int kMaxExperts = 1024;
 constexpr int kStatusNonFinite = 9; // GQ4_ERR_NONFINITE_LOGIT
 
-// Route one token with one warp.  EPL = experts per lane (>= ceil(E/32)).
+// Order-preserving key of a float (larger float -> larger unsigned key; NaN excluded).
+// Key 0 (below every float's key) marks an expert that is absent or already taken.
+__device__ __forceinline__ uint32_t route_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float route_key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Route one token with one warp.  EPL = experts per lane (>= ceil(E/32)); lane i holds
+// experts i, i+32, ...  Each of the K passes takes the largest remaining logit, the lower
+// expert index among equal logits: a warp-wide max of the lanes' best keys (redux.sync),
+// then a warp-wide min of the expert index among the lanes holding that key; only the
+// winning lane rescans its experts for its next best.
 template <int EPL>
 __device__ __forceinline__ void route_token_warp(const float *lg, int E, int K, int32_t *idx,
                                                  float *wts, int32_t *status) {
     const int lane = threadIdx.x & 31;
-    float v[EPL];
+    uint32_t key[EPL];
     bool bad = false;
     #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
-        v[i] = e < E ? lg[e] : -INFINITY;
-        if (e < E && (isnan(v[i]) || (isinf(v[i]) && v[i] > 0.f))) bad = true;
+        const float v = e < E ? lg[e] : 0.f;
+        if (e < E && (isnan(v) || (isinf(v) && v > 0.f))) bad = true;
+        // -0 and +0 compare equal: give them one key so the lower index wins their tie
+        key[i] = (e < E && !isnan(v)) ? route_key(v == 0.f ? 0.f : v) : 0u;
     }
     bad = __any_sync(0xffffffffu, bad);
-    uint32_t taken = 0;
+    // this lane's best remaining expert: the largest key, the lowest slot among equals
+    uint32_t bk = 0u;
+    int bi = 0;
+    #pragma unroll
+    for (int i = 0; i < EPL; ++i)
+        if (key[i] > bk) { bk = key[i]; bi = i; }
     float my_v[EPL];  // pick j is kept by lane j % 32 in slot j / 32 (K <= E <= 32*EPL)
     int my_e[EPL];
     #pragma unroll
     for (int i = 0; i < EPL; ++i) { my_v[i] = -INFINITY; my_e[i] = 0; }
     float vmax = -INFINITY;
     for (int j = 0; j < K; ++j) {
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
-        #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || v[i] > bv)) {
-                bv = v[i];
-                be = e;
-            }
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const int we = __reduce_min_sync(0xffffffffu, (bk == wk && wk != 0u) ? (lane + 32 * bi) : 0x7fffffff);
+        const float wv = route_key_value(wk);
+        if (we != 0x7fffffff && (we & 31) == lane) {  // the winner drops its pick
+            #pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (i == bi) key[i] = 0u;
+            bk = 0u;
+            bi = 0;
+            #pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (key[i] > bk) { bk = key[i]; bi = i; }
         }
-        #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            const bool better = (be == 0x7fffffff) ||
-                                (oe != 0x7fffffff && (ov > bv || (ov == bv && oe < be)));
-            if (better) { bv = ov; be = oe; }
-        }
-        if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
-        if (j == 0) vmax = bv;
+        if (j == 0) vmax = wv;
         if ((j & 31) == lane) {
             #pragma unroll
             for (int i = 0; i < EPL; ++i)
-                if (i == (j >> 5)) { my_v[i] = bv; my_e[i] = be; }
+                if (i == (j >> 5)) { my_v[i] = wv; my_e[i] = we; }
         }
     }
     if (!bad && isinf(vmax)) bad = true;  // no finite maximum
