@@ -153,3 +153,16 @@ def test_gate_up_general_group_size(F, H, gs, T):
     xmax = np.abs(synth.bf16_bits_to_f32(x)).max(1).astype(np.float64)
     b = h_bound(oracle.row_l1(pg, sg, H, gs), oracle.row_l1(pu, su, H, gs), xmax, g_o, u_o)
     check_bf16_close(h, h_o, b, f"gate_up gs={gs}")
+
+
+@pytest.mark.parametrize("gs,I", [(64, 256), (32, 256), (128, 512)])
+def test_matvec_rows_out_of_range_index_gives_nan(gs, I):
+    q, p, s = _packed(gs + I, 40, I, gs)
+    W = gq4.upload(p, s, gs=gs)
+    idx = np.array([0, 40, 7, -3, 39], np.int32)
+    x = synth.x_normal(2, 2, I, "bf16", 40, I, 2)
+    y = gq4.matvec_rows(W, torch.from_numpy(idx).cuda(), bf16_to_torch(x)).cpu().numpy()
+    assert np.all(np.isnan(y[:, 1])) and np.all(np.isnan(y[:, 3]))
+    ok = [0, 2, 4]
+    y_o, b = oracle.matvec_rows(p, s, idx[ok], x, gs)
+    check_close(y[:, ok], y_o, b, f"matvec_rows valid columns gs={gs}")

@@ -418,6 +418,15 @@ gq4_status launch_tc(const CUtensorMap &w0, const CUtensorMap &w1, const CUtenso
 
 }  // namespace
 
+// Group sizes the mma.sync split-K kernel also takes: 64 << k with in % 64 == 0 (a group
+// is 2^k consecutive 64-wide groups sharing one scale).  -1 when not of that form.
+int wide_group_shift(const gq4_tensor *t) {
+    if (t->in % 64) return -1;
+    for (int k = 0; k < 15; ++k)
+        if (t->gs == (64 << k)) return k;
+    return -1;
+}
+
 // ---- generic kernels (gq4_aux.cuh) ----------------------------------------------------
 // Matvec / gate+up over all rows or selected rows, any group size that is a multiple of 8.
 template <int MODE>
@@ -550,8 +559,6 @@ gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t
     if (overlap(yr, rng(x, xb)) || overlap(yr, rng(W->w, tensor_w_bytes(W))) ||
         overlap(yr, rng(W->s, tensor_s_bytes(W))))
         return GQ4_ERR_ALIAS;
-    if (check_tensor(W, 1) != GQ4_OK)  // another group size or a partial last group
-        return launch_generic<0>(W, nullptr, W->out, nullptr, x, xdt, n_tok, y, S(stream));
     SkinnyParams p{};
     p.w0 = W->w; p.s0 = W->s;
     p.O = (int)W->out; p.I = (int)W->in; p.ng = W->ng;
@@ -559,6 +566,14 @@ gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.y = y;
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    if (check_tensor(W, 1) != GQ4_OK) {  // another group size or a partial last group
+        const int sh = wide_group_shift(W);
+        if (sh < 0) return launch_generic<0>(W, nullptr, W->out, nullptr, x, xdt, n_tok, y, S(stream));
+        p.ng = (int)(W->in / 64);  // 64-wide groups; the scale of group G is column G >> sh
+        p.sng = W->ng;
+        p.gshift = sh;
+        return launch_skinny<kMatvec>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
+    }
     if (xdt == GQ4_BF16 && stream_usable(W) && (n_tok >= kBandMinCols || (W->out + 63) / 64 >= sm_count()))
         return launch_stream<kMatvec>(stream_mats(W, nullptr), p, cols, 1, nullptr, S(stream));
     if (xdt == GQ4_BF16 && n_tok >= kBandMinCols)
@@ -583,8 +598,6 @@ gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const vo
         overlap(hr, rng(Wg->w, tensor_w_bytes(Wg))) || overlap(hr, rng(Wg->s, tensor_s_bytes(Wg))) ||
         overlap(hr, rng(Wu->w, tensor_w_bytes(Wu))) || overlap(hr, rng(Wu->s, tensor_s_bytes(Wu))))
         return GQ4_ERR_ALIAS;
-    if (check_tensor(Wg, 1) != GQ4_OK || check_tensor(Wu, 1) != GQ4_OK)  // general group size
-        return launch_generic<1>(Wg, Wu, Wg->out, nullptr, x, xdt, n_tok, h, S(stream));
     SkinnyParams p{};
     p.w0 = Wg->w; p.s0 = Wg->s; p.w1 = Wu->w; p.s1 = Wu->s;
     p.O = (int)Wg->out; p.I = (int)Wg->in; p.ng = Wg->ng;
@@ -592,6 +605,14 @@ gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const vo
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.h = h;
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    if (check_tensor(Wg, 1) != GQ4_OK || check_tensor(Wu, 1) != GQ4_OK) {  // general group size
+        const int sh = wide_group_shift(Wg);
+        if (sh < 0) return launch_generic<1>(Wg, Wu, Wg->out, nullptr, x, xdt, n_tok, h, S(stream));
+        p.ng = (int)(Wg->in / 64);
+        p.sng = Wg->ng;
+        p.gshift = sh;
+        return launch_skinny<kGateUp>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
+    }
     if (xdt == GQ4_BF16 && stream_usable(Wg) && stream_usable(Wu) &&
         (n_tok >= kBandMinCols || (Wg->out + 63) / 64 >= sm_count()))
         return launch_stream<kGateUp>(stream_mats(Wg, Wu), p, cols, 1, nullptr, S(stream));
@@ -996,5 +1017,19 @@ extern "C" gq4_status gq4_matvec_rows(const gq4_tensor *W, const int32_t *idx, i
     if (overlap(yr, rng(x, (size_t)n_tok * W->in * (xdt == GQ4_F32 ? 4 : 2))) || overlap(yr, rng(idx, (size_t)n_sel * 4)) ||
         overlap(yr, rng(W->w, tensor_w_bytes(W))) || overlap(yr, rng(W->s, tensor_s_bytes(W))))
         return GQ4_ERR_ALIAS;
-    return launch_generic<0>(W, nullptr, n_sel, idx, x, xdt, n_tok, y, S(stream));
+    const int sh = wide_group_shift(W);
+    if (sh < 0) return launch_generic<0>(W, nullptr, n_sel, idx, x, xdt, n_tok, y, S(stream));
+    // group sizes 64 << sh: the mma.sync split-K kernel over 16-row tiles of the gathered rows
+    SkinnyParams p{};
+    p.w0 = W->w; p.s0 = W->s;
+    p.O = (int)W->out; p.I = (int)W->in; p.ng = (int)(W->in / 64);
+    p.sng = W->ng;
+    p.gshift = sh;
+    p.rows = idx;
+    p.n_out = (int)n_sel;
+    p.row_tiles = (int)((n_sel + 15) / 16);
+    p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
+    p.y = y;
+    const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
+    return launch_skinny<kMatvec>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
 }

@@ -56,6 +56,13 @@ struct SkinnyParams {
     const float *wts;
     float *zero_ptr;    // moe gate-up: y zeroed here before the down kernel adds into it
     int64_t zero_n;     // floats (multiple of 4)
+    // split-K kernel, plain matvec / gate+up only: a group size of 64 << gshift (scale of
+    // 64-wide group G at column G >> gshift of a scale row of sng floats; 0 = ng), and an
+    // optional gather list: output j < n_out is weight row rows[j]
+    int gshift;
+    int sng;
+    const int32_t *rows;
+    int n_out;
 };
 
 template <int MODE>
@@ -146,6 +153,8 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
 
     const int n_units = TR::kMoe ? (*p.n_active) * p.row_tiles : p.row_tiles;
     const int gb = (warp * p.ng) >> 3, ge = ((warp + 1) * p.ng) >> 3;
+    const int sng = p.sng ? p.sng : p.ng;          // scales per weight row
+    const int n_out = p.rows ? p.n_out : p.O;      // output rows
     int staged_e = -1, staged_c0 = -1;
 
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
@@ -163,8 +172,14 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
         const float *S0 = p.s0 + (int64_t)e * p.estride_s;
         const uint8_t *W1 = PAIR == 2 ? p.w1 + (int64_t)e * p.estride_w : nullptr;
         const float *S1 = PAIR == 2 ? p.s1 + (int64_t)e * p.estride_s : nullptr;
-        const int rA = rt * 16 + g, rB = rA + 8;
-        const bool vA = rA < p.O, vB = rB < p.O;
+        // output rows jA, jB of this lane; their weight rows (gathered or the same)
+        const int jA = rt * 16 + g, jB = jA + 8;
+        int rA = jA, rB = jB;
+        if (!TR::kMoe && p.rows) {
+            rA = jA < n_out ? p.rows[jA] : -1;
+            rB = jB < n_out ? p.rows[jB] : -1;
+        }
+        const bool vA = jA < n_out && rA >= 0 && rA < p.O, vB = jB < n_out && rB >= 0 && rB < p.O;
 
         for (int c0 = 0; c0 < cols; c0 += p.xcols) {
             const int nc = min(p.xcols, cols - c0);
@@ -201,8 +216,8 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
                             const int64_t off = (int64_t)G * 32 + t * 8;
                             wa[m][q] = (ok && vA) ? ldg_stream_u2(Wm + (int64_t)rA * rb + off) : make_uint2(0, 0);
                             wb[m][q] = (ok && vB) ? ldg_stream_u2(Wm + (int64_t)rB * rb + off) : make_uint2(0, 0);
-                            sa[m][q] = (ok && vA) ? ldg_f32(Sm + (int64_t)rA * p.ng + G) : 0.f;
-                            sb[m][q] = (ok && vB) ? ldg_f32(Sm + (int64_t)rB * p.ng + G) : 0.f;
+                            sa[m][q] = (ok && vA) ? ldg_f32(Sm + (int64_t)rA * sng + (G >> p.gshift)) : 0.f;
+                            sb[m][q] = (ok && vB) ? ldg_f32(Sm + (int64_t)rB * sng + (G >> p.gshift)) : 0.f;
                         }
                     }
                     #pragma unroll
@@ -266,7 +281,7 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
                     for (int i = threadIdx.x; i < 16 * ntok; i += blockDim.x) {
                         const int row = i & 15, tl = i >> 4;
                         const int o = rt * 16 + row;
-                        if (o >= p.O) continue;
+                        if (o >= n_out) continue;
                         const int tok = (c0 + cc) / 3 + tl;
                         float v[PAIR];
                         #pragma unroll
@@ -277,16 +292,17 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
                                     s += red[((w * PAIR + m) * 16 + row) * NCOL + tl * 3 + sp];
                             v[m] = s;
                         }
+                        if (p.rows && (p.rows[o] < 0 || p.rows[o] >= p.O)) v[0] = __uint_as_float(0x7fc00000u);
                         if (MODE == kMatvec)
-                            p.y[(int64_t)tok * p.O + o] = v[0];
+                            p.y[(int64_t)tok * n_out + o] = v[0];
                         else
-                            ((float *)p.h)[(int64_t)tok * p.O + o] = silu_mul(v[0], v[PAIR - 1]);
+                            ((float *)p.h)[(int64_t)tok * n_out + o] = silu_mul(v[0], v[PAIR - 1]);
                     }
                 } else {
                     for (int i = threadIdx.x; i < 16 * ncc; i += blockDim.x) {
                         const int row = i & 15, cl = i >> 4;
                         const int o = rt * 16 + row;
-                        if (o >= p.O) continue;
+                        if (o >= n_out) continue;
                         float v[PAIR];
                         #pragma unroll
                         for (int m = 0; m < PAIR; ++m) {
@@ -295,10 +311,12 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
                             v[m] = s;
                         }
                         const int c = c0 + cc + cl;
+                        if (!TR::kMoe && p.rows && (p.rows[o] < 0 || p.rows[o] >= p.O))
+                            v[0] = __uint_as_float(0x7fc00000u);
                         if (MODE == kMatvec) {
-                            p.y[(int64_t)c * p.O + o] = v[0];
+                            p.y[(int64_t)c * n_out + o] = v[0];
                         } else if (MODE == kGateUp) {
-                            ((uint16_t *)p.h)[(int64_t)c * p.O + o] = (uint16_t)bf16_bits_rn(silu_mul(v[0], v[1]));
+                            ((uint16_t *)p.h)[(int64_t)c * n_out + o] = (uint16_t)bf16_bits_rn(silu_mul(v[0], v[1]));
                         } else if (MODE == kMoeGateUp) {
                             ((uint16_t *)p.h)[(int64_t)(row0 + c) * p.O + o] = (uint16_t)bf16_bits_rn(silu_mul(v[0], v[1]));
                         } else {  // kMoeDown: weighted scatter-add into y
