@@ -84,6 +84,10 @@ def lib() -> ctypes.CDLL:
         L.orc_dequant_rows.argtypes = [P, P, I64, I64, I64, P, I64, P, I, P]
         L.orc_dequant_rows.restype = None
         L.orc_matvec_rows.argtypes = [P, P, I64, I64, I64, P, I64, P, I, I64, P, P]
+        L.orc_mla_absorb_q.argtypes = [P, P, I64, I64, I64, I64, I64, P, I, I64, P, P]
+        L.orc_mla_absorb_q.restype = None
+        L.orc_mla_absorb_v.argtypes = [P, P, I64, I64, I64, I64, I64, P, I, I64, P, P]
+        L.orc_mla_absorb_v.restype = None
         L.orc_matvec_rows.restype = None
     return _lib
 
@@ -299,3 +303,29 @@ def matvec_rows(packed, scales, idx, x, gs: int = 64):
     lib().orc_matvec_rows(_p(packed), _p(scales), packed.shape[0], I, gs, _p(idx), n, _p(x),
                           _xdt(x), T, _p(y), _p(b))
     return y, b
+
+
+def _mla(fn, packed, scales, R, nh, dn, dv, x, width, gs):
+    packed = _c(packed, np.uint8)
+    scales = _c(scales, np.float32)
+    x = np.ascontiguousarray(x)
+    assert packed.shape[0] == nh * (dn + dv) and x.shape[-2:] == (nh, width), (packed.shape, x.shape)
+    T = x.shape[0]
+    n_out = R if fn == "q" else dv
+    y = np.empty((T, nh, n_out), np.float64)
+    b = np.empty((T, nh, n_out), np.float64)
+    f = lib().orc_mla_absorb_q if fn == "q" else lib().orc_mla_absorb_v
+    f(_p(packed), _p(scales), R, gs, nh, dn, dv, _p(x), _xdt(x), T, _p(y), _p(b))
+    return y, b
+
+
+def mla_absorb_q(packed, scales, R, nh, dn, dv, q_nope, gs: int = 64):
+    """q_lat [T][nh][R] fp64 = sum_d q_nope[t][h][d] * w(h*(dn+dv)+d, c), and its bound.
+    q_nope [T][nh][dn] f32 or bf16 bits (uint16)."""
+    return _mla("q", packed, scales, R, nh, dn, dv, q_nope, dn, gs)
+
+
+def mla_absorb_v(packed, scales, R, nh, dn, dv, lat, gs: int = 64):
+    """o [T][nh][dv] fp64 = sum_c lat[t][h][c] * w(h*(dn+dv)+dn+v, c), and its bound.
+    lat [T][nh][R] f32 or bf16 bits (uint16)."""
+    return _mla("v", packed, scales, R, nh, dn, dv, lat, R, gs)

@@ -18,9 +18,11 @@
  *   [PXQ]    pxq_llama.cpp release notes 2026-09-02.
  * Where the pages are silent the reading is stated at the function.
  *
- * Pins (tests/test_oracle.py): every function here is checked against hand-worked
- * nibble tables, closed forms, the fmt=2 identity, brute-force sorting and the worked
- * size example of the kv_b tensor; none of its results is compared with itself.
+ * Pins (tests/test_oracle.py, tests/test_oracle_next.py): every function here is checked
+ * against hand-worked nibble and rounding tables, closed forms, the fmt=2 identity,
+ * exact integer arithmetic, brute-force sorting, an independent numpy decode and the
+ * worked size examples of the kv_b tensor and the expert; none of its results is
+ * compared with itself.
  */
 #include <math.h>
 #include <stdint.h>
@@ -447,6 +449,67 @@ void orc_matvec_rows(const uint8_t *packed, const float *scales, int64_t O, int6
             }
             y[t * n + j] = acc;
             if (bound) bound[t * n + j] = l1 * xmax;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------------
+ * Grouped-scale MLA absorb projections over the kv_b tensor.
+ * [PR298] "fmt=4 CUDA attention crash — root cause": the Q- and V-projection loops of
+ * the two MLA attention absorb kernels multiply weights of the kv_b tensor (28,672 rows
+ * x 512 inputs, 8 groups of 64 per row) by their scale.  With fmt=4 the scale of weight
+ * (row, k) is scales[row*ng + k/gs], looked up inside the accumulation loop; one scale
+ * per row applied after the loop is the fmt=2 rule and is wrong here.
+ * Reading (the pages name the kernels, not their shapes): the rows of kv_b come in
+ * per-head blocks of dn + dv rows, the first dn the key part and the last dv the value
+ * part; the inputs are the R latent channels.  With D = dn + dv:
+ *   Q absorb: q_lat[t][h][c] = sum_{d<dn} q_nope[t][h][d] * w(h*D + d, c),      c < R
+ *   V absorb: o[t][h][v]     = sum_{c<R}  lat[t][h][c]   * w(h*D + dn + v, c),  v < dv
+ * fp64, natural summation order.  bound = sum |w| * max |input| over the summed index
+ * (the Sigma|terms| scale of the acceptance test).
+ * ------------------------------------------------------------------------------- */
+void orc_mla_absorb_q(const uint8_t *packed, const float *scales, int64_t R, int64_t gs,
+                      int64_t nh, int64_t dn, int64_t dv, const void *q, int qdt, int64_t T,
+                      double *out, double *bound)
+{
+    int64_t D = dn + dv, O = nh * D;
+#pragma omp parallel for schedule(static)
+    for (int64_t th = 0; th < T * nh; th++) {
+        int64_t h = th % nh;
+        for (int64_t c = 0; c < R; c++) {
+            double acc = 0.0, l1 = 0.0, qmax = 0.0;
+            for (int64_t d = 0; d < dn; d++) {
+                double w = orc_weight(packed, scales, O, R, gs, h * D + d, c);
+                double qv = orc_x(q, qdt, th * dn + d);
+                acc += qv * w;
+                l1 += fabs(w);
+                if (fabs(qv) > qmax) qmax = fabs(qv);
+            }
+            out[th * R + c] = acc;
+            if (bound) bound[th * R + c] = l1 * qmax;
+        }
+    }
+}
+
+void orc_mla_absorb_v(const uint8_t *packed, const float *scales, int64_t R, int64_t gs,
+                      int64_t nh, int64_t dn, int64_t dv, const void *lat, int ldt, int64_t T,
+                      double *out, double *bound)
+{
+    int64_t D = dn + dv, O = nh * D;
+#pragma omp parallel for schedule(static)
+    for (int64_t th = 0; th < T * nh; th++) {
+        int64_t h = th % nh;
+        for (int64_t v = 0; v < dv; v++) {
+            double acc = 0.0, l1 = 0.0, xmax = 0.0;
+            for (int64_t c = 0; c < R; c++) {
+                double w = orc_weight(packed, scales, O, R, gs, h * D + dn + v, c);
+                double xv = orc_x(lat, ldt, th * R + c);
+                acc += xv * w;
+                l1 += fabs(w);
+                if (fabs(xv) > xmax) xmax = fabs(xv);
+            }
+            out[th * dv + v] = acc;
+            if (bound) bound[th * dv + v] = l1 * xmax;
         }
     }
 }

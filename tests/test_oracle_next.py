@@ -166,3 +166,102 @@ def test_matvec_rows_vs_numpy(O, I, gs, T):
     ref = x.astype(np.float64) @ dense[idx].T
     assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
     assert np.all(np.abs(y) <= b * (1 + 1e-12))
+
+
+# ---------------------------------------------------------------- MLA absorb projections
+def _mla_tensor(nh, dn, dv, R, gs, seed, pow2=False):
+    """kv_b-like tensor: nh blocks of dn key rows + dv value rows, R inputs."""
+    rng = np.random.default_rng(seed)
+    O = nh * (dn + dv)
+    q = rng.integers(-8, 8, size=(O, R)).astype(np.int8)
+    ng = -(-R // gs)
+    if pow2:
+        scales = (2.0 ** rng.integers(-6, 2, size=(O, ng))).astype(np.float32)
+    else:
+        scales = rng.uniform(0.002, 0.02, size=(O, ng)).astype(np.float32)
+    return q, oracle.pack(q), scales
+
+
+@pytest.mark.parametrize("nh,dn,dv,R,gs,T", [(2, 3, 5, 128, 64, 1), (3, 16, 8, 96, 64, 2),
+                                             (1, 4, 4, 40, 16, 3), (2, 8, 16, 512, 64, 2)])
+def test_mla_absorb_vs_numpy(nh, dn, dv, R, gs, T):
+    """Both projections against an independent decode and einsum over the head blocks
+    (partial last group in the 96- and 40-wide cases)."""
+    _, packed, scales = _mla_tensor(nh, dn, dv, R, gs, seed=nh * 100 + R)
+    W = _np_dequant(packed, scales, R, gs).reshape(nh, dn + dv, R)
+    rng = np.random.default_rng(R)
+    qn = rng.standard_normal((T, nh, dn)).astype(np.float32)
+    lat = rng.standard_normal((T, nh, R)).astype(np.float32)
+    got_q, b_q = oracle.mla_absorb_q(packed, scales, R, nh, dn, dv, qn, gs)
+    ref_q = np.einsum("thd,hdc->thc", qn.astype(np.float64), W[:, :dn, :])
+    np.testing.assert_allclose(got_q, ref_q, rtol=1e-12, atol=1e-12 * np.abs(ref_q).max())
+    assert np.all(np.abs(ref_q) <= b_q * (1 + 1e-12))
+    got_v, b_v = oracle.mla_absorb_v(packed, scales, R, nh, dn, dv, lat, gs)
+    ref_v = np.einsum("thc,hvc->thv", lat.astype(np.float64), W[:, dn:, :])
+    np.testing.assert_allclose(got_v, ref_v, rtol=1e-12, atol=1e-12 * np.abs(ref_v).max())
+    assert np.all(np.abs(ref_v) <= b_v * (1 + 1e-12))
+
+
+def test_mla_absorb_exact_integer_arithmetic():
+    """Power-of-two scales and integer inputs: every product and partial sum is exact in
+    fp64, so the results equal integer arithmetic done in Python."""
+    nh, dn, dv, R, gs, T = 2, 5, 3, 80, 16, 2
+    q, packed, scales = _mla_tensor(nh, dn, dv, R, gs, seed=5, pow2=True)
+    rng = np.random.default_rng(6)
+    qn = rng.integers(-4, 5, size=(T, nh, dn)).astype(np.float32)
+    lat = rng.integers(-4, 5, size=(T, nh, R)).astype(np.float32)
+    got_q, _ = oracle.mla_absorb_q(packed, scales, R, nh, dn, dv, qn, gs)
+    got_v, _ = oracle.mla_absorb_v(packed, scales, R, nh, dn, dv, lat, gs)
+    D = dn + dv
+    for t in range(T):
+        for h in range(nh):
+            for c in range(R):
+                want = sum(int(qn[t, h, d]) * int(q[h * D + d, c]) * float(scales[h * D + d, c // gs])
+                           for d in range(dn))
+                assert got_q[t, h, c] == want
+            for v in range(dv):
+                r = h * D + dn + v
+                want = sum(int(lat[t, h, c]) * int(q[r, c]) * float(scales[r, c // gs]) for c in range(R))
+                assert got_v[t, h, v] == want
+
+
+def test_mla_absorb_q_one_hot_reads_the_group_scale():
+    """A one-hot q_nope on (head h, key row d) returns that kv_b row exactly, with the
+    scale of each column's own group; one scale per row (the fmt=2 rule the pages' crash
+    came from) gives a different row."""
+    nh, dn, dv, R, gs = 3, 4, 2, 256, 64
+    q, packed, scales = _mla_tensor(nh, dn, dv, R, gs, seed=9, pow2=True)
+    scales[:, 1] *= 2.0  # make sure neighbouring groups of a row differ
+    h, d = 2, 3
+    row = h * (dn + dv) + d
+    qn = np.zeros((1, nh, dn), np.float32)
+    qn[0, h, d] = 1.0
+    got, _ = oracle.mla_absorb_q(packed, scales, R, nh, dn, dv, qn, gs)
+    want = scales[row, np.arange(R) // gs].astype(np.float64) * q[row].astype(np.float64)
+    assert np.array_equal(got[0, h], want)
+    assert not np.any(got[0, [0, 1]])
+    per_row = scales.reshape(-1)[row] * q[row].astype(np.float64)  # wscale[row] on an O*ng buffer
+    assert not np.array_equal(got[0, h], per_row)
+
+
+def test_mla_absorb_v_one_hot_and_fmt2_identity():
+    """A one-hot latent channel c returns column c of each head's value rows; with all
+    group scales of a row equal, the V projection is the per-row (fmt=2) product."""
+    nh, dn, dv, R, gs = 2, 3, 4, 128, 64
+    q, packed, scales = _mla_tensor(nh, dn, dv, R, gs, seed=11, pow2=True)
+    c = 77
+    lat = np.zeros((1, nh, R), np.float32)
+    lat[0, :, c] = 1.0
+    got, _ = oracle.mla_absorb_v(packed, scales, R, nh, dn, dv, lat, gs)
+    D = dn + dv
+    for h in range(nh):
+        rows = h * D + dn + np.arange(dv)
+        assert np.array_equal(got[0, h], scales[rows, c // gs].astype(np.float64) * q[rows, c])
+    flat = np.repeat(scales[:, :1], scales.shape[1], axis=1)  # one scale per row
+    rng = np.random.default_rng(12)
+    lat = rng.integers(-3, 4, size=(2, nh, R)).astype(np.float32)
+    got, _ = oracle.mla_absorb_v(packed, flat, R, nh, dn, dv, lat, gs)
+    for h in range(nh):
+        rows = h * D + dn + np.arange(dv)
+        want = flat[rows, 0].astype(np.float64)[None] * (lat[:, h].astype(np.int64) @ q[rows].T.astype(np.int64))
+        assert np.array_equal(got[:, h], want)
