@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define GQ4_ABI_VERSION 2u
+#define GQ4_ABI_VERSION 3u
 
 typedef struct CUstream_st *gq4_stream_t; /* binary-compatible with cudaStream_t */
 typedef struct CUevent_st *gq4_event_t;   /* binary-compatible with cudaEvent_t */
@@ -265,6 +265,29 @@ gq4_status gq4_dequant_rows(const gq4_tensor *W, const int32_t *idx, int64_t n,
 gq4_status gq4_matvec_rows(const gq4_tensor *W, const int32_t *idx, int64_t n_sel,
                            const void *x, gq4_dtype xdt, int64_t n_tok, float *y,
                            gq4_stream_t stream);
+
+/* ---- grouped-scale MLA absorb projections over the kv_b tensor
+ * colibri PR #298, "fmt=4 CUDA attention crash — root cause": the Q- and V-projection
+ * loops of the MLA attention absorb kernels multiply kv_b weights by their scale, and
+ * with fmt=4 the scale of weight (row, k) is scales[row*ng + k/gs], looked up inside the
+ * accumulation loop (one scale per row, the fmt=2 rule, reads the wrong entries of the
+ * O*ng scale array).  These calls run the two projections on their own.
+ *   W: the kv_b tensor, out = n_heads * (d_nope + d_v) rows in per-head blocks (d_nope
+ *      key rows, then d_v value rows), in = R latent channels; any gs % 8 == 0 with
+ *      R % 8 == 0, R <= 2048, d_nope <= 1024 (GQ4_ERR_UNSUPPORTED beyond); the first
+ *      expert of a stacked tensor is used.  With D = d_nope + d_v:
+ * gq4_mla_absorb_q: q_lat[t][h][c] = sum_{d < d_nope} q_nope[t][h][d] * w(h*D + d, c)
+ *      q_nope: device [T][n_heads][d_nope] of qdt (GQ4_F32 or GQ4_BF16);
+ *      q_lat: device f32 [T][n_heads][R].
+ * gq4_mla_absorb_v: o[t][h][v] = sum_{c < R} lat[t][h][c] * w(h*D + d_nope + v, c)
+ *      lat: device [T][n_heads][R] of ldt; o: device f32 [T][n_heads][d_v].
+ * fp32 accumulation.  T <= 262140.  Outputs must not overlap the inputs or W. */
+gq4_status gq4_mla_absorb_q(const gq4_tensor *W, int32_t n_heads, int32_t d_nope, int32_t d_v,
+                            const void *q_nope, gq4_dtype qdt, int64_t T, float *q_lat,
+                            gq4_stream_t stream);
+gq4_status gq4_mla_absorb_v(const gq4_tensor *W, int32_t n_heads, int32_t d_nope, int32_t d_v,
+                            const void *lat, gq4_dtype ldt, int64_t T, float *o,
+                            gq4_stream_t stream);
 
 /* moe_expert_ffn_noalloc: the same layer as moe_expert_ffn, for callers that cannot
  * allocate device memory -- a plug-in whose host program owns every device allocation

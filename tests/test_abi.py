@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = gq4.lib()
-    assert lib.gq4_abi_version() == 2
+    assert lib.gq4_abi_version() == 3
     for st in range(10):
         assert lib.gq4_status_string(st).decode()
     assert lib.gq4_status_string(77) == b"unknown status"
@@ -184,3 +184,25 @@ def test_quantize_and_row_ops_argument_checks():
     assert mr(xdt=5) == gq4.ERR_UNSUPPORTED
     assert mr(y=0x700000) == gq4.ERR_ALIAS
     assert mr(idx=0x500002) == gq4.ERR_ALIGN
+
+
+def test_mla_absorb_argument_checks():
+    """Rejected MLA absorb calls return before anything is launched (fake pointers)."""
+    L = gq4.lib()
+    W = _desc(out=2 * (16 + 48), in_=512)
+    for fn in (L.gq4_mla_absorb_q, L.gq4_mla_absorb_v):
+        c = lambda nh=2, dn=16, dv=48, x=0x700000, dt=1, T=3, out=0x900000, d=W: \
+            fn(ctypes.byref(d), nh, dn, dv, x, dt, T, out, None)
+        assert c(x=0) == gq4.ERR_NULL
+        assert c(out=0) == gq4.ERR_NULL
+        assert c(dv=47) == gq4.ERR_SHAPE           # n_heads * (d_nope + d_v) != out
+        assert c(nh=0) == gq4.ERR_SHAPE
+        assert c(T=0) == gq4.ERR_SHAPE
+        assert c(T=4 * 65536) == gq4.ERR_SHAPE
+        assert c(dt=7) == gq4.ERR_UNSUPPORTED
+        assert c(d=_desc(out=2 * (16 + 48), in_=4096)) == gq4.ERR_UNSUPPORTED  # R > 2048
+        assert c(dn=1040, dv=-976) == gq4.ERR_SHAPE
+        assert c(x=0x700004) == gq4.ERR_ALIGN
+        assert c(out=0x700000) == gq4.ERR_ALIAS
+    big = _desc(out=1025 + 7, in_=64)
+    assert L.gq4_mla_absorb_q(ctypes.byref(big), 1, 1025, 7, 0x700000, 0, 1, 0x900000, None) == gq4.ERR_UNSUPPORTED

@@ -166,3 +166,42 @@ def test_matvec_rows_out_of_range_index_gives_nan(gs, I):
     ok = [0, 2, 4]
     y_o, b = oracle.matvec_rows(p, s, idx[ok], x, gs)
     check_close(y[:, ok], y_o, b, f"matvec_rows valid columns gs={gs}")
+
+
+# ---------------------------------------------------------------- MLA absorb projections
+def _kvb(seed, nh, dn, dv, R, gs):
+    O = nh * (dn + dv)
+    packed = synth.packed_uniform(seed, O, R, 3)
+    scales = synth.scales_uniform(seed, O, -(-R // gs), 0.002, 0.02, 3)
+    return packed, scales
+
+
+def _act(seed, shape, dt):
+    x = synth.rng(seed, 5).standard_normal(shape).astype(np.float32)
+    if dt == "bf16":
+        xb = synth.to_bf16_bits(x)
+        return xb, bf16_to_torch(xb)
+    return x, torch.from_numpy(x).cuda()
+
+
+@pytest.mark.parametrize("nh,dn,dv,R,gs,T,dt", [
+    (64, 192, 256, 512, 64, 1, "bf16"),   # the pages' kv_b: 28,672 rows x 512, 8 groups per row
+    (64, 192, 256, 512, 64, 5, "f32"),    # two token blocks, the second ragged
+    (3, 5, 7, 40, 16, 6, "f32"),          # partial last group (40 = 16 + 16 + 8)
+    (2, 9, 33, 24, 16, 3, "bf16"),        # value rows spill into a second block row range
+    (4, 16, 8, 1024, 128, 2, "bf16"),     # 128 words per row: two key-row splits
+    (2, 12, 20, 2048, 64, 4, "f32"),      # 256 words per row: one thread per word
+    (1, 1, 1, 8, 8, 1, "f32"),            # one word, one group
+])
+def test_mla_absorb_q_and_v(nh, dn, dv, R, gs, T, dt):
+    packed, scales = _kvb(nh * 1000 + R + gs, nh, dn, dv, R, gs)
+    W = gq4.upload(packed, scales, gs=gs)
+    qn_h, qn = _act(R + T, (T, nh, dn), dt)
+    lat_h, lat = _act(R + T + 1, (T, nh, R), dt)
+    q_lat = gq4.mla_absorb_q(W, nh, dn, dv, qn)
+    o = gq4.mla_absorb_v(W, nh, dn, dv, lat)
+    torch.cuda.synchronize()
+    ref_q, b_q = oracle.mla_absorb_q(packed, scales, R, nh, dn, dv, qn_h, gs)
+    ref_v, b_v = oracle.mla_absorb_v(packed, scales, R, nh, dn, dv, lat_h, gs)
+    check_close(q_lat.cpu().numpy(), ref_q, b_q, "mla absorb q")
+    check_close(o.cpu().numpy(), ref_v, b_v, "mla absorb v")

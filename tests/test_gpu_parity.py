@@ -233,6 +233,8 @@ def _toy(T, E, K, H=128, F=128, seed=3, **kw):
                                        # the decode path, multi-pass experts (> 192 rows)
                                        (64, 4, 2, 256, 128), (40, 8, 4, 384, 192), (300, 2, 1, 128, 64),
                                        (500, 2, 2, 128, 128), (48, 4, 2, 192, 128), (130, 6, 3, 512, 256),
+                                       # passes of many sizes in one CTA (activation byte ring laps)
+                                       (600, 12, 3, 256, 128), (1000, 8, 2, 128, 64),
                                        # TMA-fed decode kernel for gate+up and down (H, F multiples
                                        # of 256), alone and beside the tensor-core path
                                        (12, 16, 4, 256, 256), (30, 8, 8, 512, 256), (20, 64, 8, 256, 512),

@@ -12,6 +12,7 @@
 #include "gq4.h"
 #include "gq4_aux.cuh"
 #include "gq4_common.cuh"
+#include "gq4_mla.cuh"
 #include "gq4_route.cuh"
 #include "gq4_skinny.cuh"
 #include "gq4_stream.cuh"
@@ -1032,4 +1033,73 @@ extern "C" gq4_status gq4_matvec_rows(const gq4_tensor *W, const int32_t *idx, i
     p.y = y;
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
     return launch_skinny<kMatvec>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
+}
+
+// ---------------------------------------------------------------------------------------
+// Grouped-scale MLA absorb projections over the kv_b tensor
+// ---------------------------------------------------------------------------------------
+namespace {
+gq4_status mla_check(const gq4_tensor *W, int32_t nh, int32_t dn, int32_t dv, int64_t T, const void *in,
+                     gq4_dtype dt, const float *out) {
+    gq4_status st = check_tensor_generic(W, 1);
+    if (st != GQ4_OK) return st;
+    if (!in || !out) return GQ4_ERR_NULL;
+    if (dt != GQ4_F32 && dt != GQ4_BF16) return GQ4_ERR_UNSUPPORTED;
+    if (nh < 1 || dn < 1 || dv < 1 || T < 1) return GQ4_ERR_SHAPE;
+    if ((int64_t)nh * ((int64_t)dn + dv) != W->out) return GQ4_ERR_SHAPE;
+    if ((T + kMlaTok - 1) / kMlaTok > 65535) return GQ4_ERR_SHAPE;
+    if (W->in > kMlaMaxR || dn > kMlaMaxDn) return GQ4_ERR_UNSUPPORTED;
+    if (!aligned16(in) || !aligned16(out)) return GQ4_ERR_ALIGN;
+    return GQ4_OK;
+}
+}  // namespace
+
+extern "C" gq4_status gq4_mla_absorb_q(const gq4_tensor *W, int32_t n_heads, int32_t d_nope, int32_t d_v,
+                                       const void *q_nope, gq4_dtype qdt, int64_t T, float *q_lat,
+                                       gq4_stream_t stream) {
+    gq4_status st = mla_check(W, n_heads, d_nope, d_v, T, q_nope, qdt, q_lat);
+    if (st != GQ4_OK) return st;
+    const int R = (int)W->in;
+    const Range o = rng(q_lat, (size_t)T * n_heads * R * 4);
+    if (overlap(o, rng(q_nope, (size_t)T * n_heads * d_nope * (qdt == GQ4_F32 ? 4 : 2))) ||
+        overlap(o, rng(W->w, tensor_w_bytes(W))) || overlap(o, rng(W->s, tensor_s_bytes(W))))
+        return GQ4_ERR_ALIAS;
+    const int words = R / 8;
+    const int nsplit = words >= kMlaThreads ? 1 : kMlaThreads / words;
+    const int threads = words >= kMlaThreads ? kMlaThreads : words * nsplit;
+    const size_t smem = ((size_t)kMlaTok * d_nope + (nsplit > 1 ? (size_t)nsplit * kMlaTok * R : 0)) * 4;
+    const dim3 grid((unsigned)n_heads, (unsigned)((T + kMlaTok - 1) / kMlaTok));
+    cudaStream_t s = S(stream);
+    if (qdt == GQ4_F32)
+        gq4_mla_q_kernel<0><<<grid, threads, smem, s>>>((const uint32_t *)W->w, W->s, R, W->ng, W->gs, n_heads,
+                                                        d_nope, d_v, q_nope, T, q_lat);
+    else
+        gq4_mla_q_kernel<1><<<grid, threads, smem, s>>>((const uint32_t *)W->w, W->s, R, W->ng, W->gs, n_heads,
+                                                        d_nope, d_v, q_nope, T, q_lat);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}
+
+extern "C" gq4_status gq4_mla_absorb_v(const gq4_tensor *W, int32_t n_heads, int32_t d_nope, int32_t d_v,
+                                       const void *lat, gq4_dtype ldt, int64_t T, float *o,
+                                       gq4_stream_t stream) {
+    gq4_status st = mla_check(W, n_heads, d_nope, d_v, T, lat, ldt, o);
+    if (st != GQ4_OK) return st;
+    const int R = (int)W->in;
+    const Range orng = rng(o, (size_t)T * n_heads * d_v * 4);
+    if (overlap(orng, rng(lat, (size_t)T * n_heads * R * (ldt == GQ4_F32 ? 4 : 2))) ||
+        overlap(orng, rng(W->w, tensor_w_bytes(W))) || overlap(orng, rng(W->s, tensor_s_bytes(W))))
+        return GQ4_ERR_ALIAS;
+    const int rows_per_block = (kMlaThreads / 32) * kMlaVRowsPerWarp;
+    const dim3 grid((unsigned)n_heads, (unsigned)((d_v + rows_per_block - 1) / rows_per_block),
+                    (unsigned)((T + kMlaTok - 1) / kMlaTok));
+    if (grid.y > 65535) return GQ4_ERR_SHAPE;
+    const size_t smem = (size_t)kMlaTok * R * 4;
+    cudaStream_t s = S(stream);
+    if (ldt == GQ4_F32)
+        gq4_mla_v_kernel<0><<<grid, kMlaThreads, smem, s>>>((const uint32_t *)W->w, W->s, R, W->ng, W->gs,
+                                                            n_heads, d_nope, d_v, lat, T, o);
+    else
+        gq4_mla_v_kernel<1><<<grid, kMlaThreads, smem, s>>>((const uint32_t *)W->w, W->s, R, W->ng, W->gs,
+                                                            n_heads, d_nope, d_v, lat, T, o);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
 }

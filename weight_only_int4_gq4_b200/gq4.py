@@ -16,7 +16,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgq4.so")
-ABI_VERSION = 2
+ABI_VERSION = 3
 MOE_STAGE_EVENTS = 6
 MOE_LARGE_MIN_ROWS = 33  # GQ4_MOE_LARGE_MIN_ROWS
 NOALLOC_SCRATCH_BYTES = 16 << 20  # GQ4_NOALLOC_SCRATCH_BYTES
@@ -72,6 +72,8 @@ _SIGS = {
     "gq4_quantize": ([_P, _I64, _I64, _I32, _P, _SZ, _P, _SZ, _P, _TP], ctypes.c_int),
     "gq4_dequant_rows": ([_TP, _P, _I64, _P, _I32, _P, ctypes.c_int, _P], ctypes.c_int),
     "gq4_matvec_rows": ([_TP, _P, _I64, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
+    "gq4_mla_absorb_q": ([_TP, _I32, _I32, _I32, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
+    "gq4_mla_absorb_v": ([_TP, _I32, _I32, _I32, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -387,3 +389,29 @@ def matvec_rows(W: Tensor, idx: torch.Tensor, x: torch.Tensor, y: torch.Tensor |
     _check(_lib.gq4_matvec_rows(W.ref(), idx.data_ptr(), n, x.data_ptr(), _xdt(x), x.shape[0], y.data_ptr(),
                                 _stream(stream)), "gq4_matvec_rows")
     return y
+
+
+def mla_absorb_q(W: Tensor, n_heads: int, d_nope: int, d_v: int, q_nope: torch.Tensor,
+                 q_lat: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """q_lat [T][n_heads][R] f32 = q_nope [T][n_heads][d_nope] times each head's key rows
+    of the kv_b tensor W (rows in per-head blocks of d_nope key + d_v value rows)."""
+    T = q_nope.shape[0]
+    if q_lat is None:
+        q_lat = torch.empty(T, n_heads, W.in_, dtype=torch.float32, device=q_nope.device)
+    _need_cuda(q_nope, q_lat)
+    _check(_lib.gq4_mla_absorb_q(W.ref(), n_heads, d_nope, d_v, q_nope.data_ptr(), _xdt(q_nope), T,
+                                 q_lat.data_ptr(), _stream(stream)), "gq4_mla_absorb_q")
+    return q_lat
+
+
+def mla_absorb_v(W: Tensor, n_heads: int, d_nope: int, d_v: int, lat: torch.Tensor,
+                 o: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """o [T][n_heads][d_v] f32 = lat [T][n_heads][R] times each head's value rows of the
+    kv_b tensor W."""
+    T = lat.shape[0]
+    if o is None:
+        o = torch.empty(T, n_heads, d_v, dtype=torch.float32, device=lat.device)
+    _need_cuda(lat, o)
+    _check(_lib.gq4_mla_absorb_v(W.ref(), n_heads, d_nope, d_v, lat.data_ptr(), _xdt(lat), T,
+                                 o.data_ptr(), _stream(stream)), "gq4_mla_absorb_v")
+    return o

@@ -13,7 +13,9 @@ seeded synthetic data with the shapes of the workloads:
   * quantisation of f32 weights (a 6144x2048 expert, a 151936x4096 matrix);
   * row gather of 512 rows of a 151936x4096 matrix to bf16 (embedding lookup);
   * matvec over 512 selected rows of that matrix;
-  * general group size: a 14336x4096 matvec with gs = 128.
+  * general group size: a 14336x4096 matvec with gs = 128;
+  * the MLA absorb projections over a 28672x512 kv_b tensor (64 heads of 192 key and
+    256 value rows), 1 and 32 tokens.
 """
 from __future__ import annotations
 
@@ -142,6 +144,21 @@ def main():
         y = torch.empty(1, O, device=dev)
         ms = time_graph(lambda: gq4.matvec(W, x, y), args.reps, flush)
         report("matvec_gs128_14336x4096_t1", ms, wbytes(O, I, 128) + I * 2 + O * 4, peak)
+
+    if want("mla_absorb"):
+        # the pages' kv_b tensor: 28,672 rows x 512 latent inputs, read as 64 heads of
+        # 192 key + 256 value rows
+        nh, dn, dv, R = 64, 192, 256, 512
+        W = rand_tensor(nh * (dn + dv), R, seed=31)
+        for T in (1, 32):
+            qn = torch.randn(T, nh, dn, device=dev).to(torch.bfloat16)
+            lat = torch.randn(T, nh, R, device=dev).to(torch.bfloat16)
+            ql = torch.empty(T, nh, R, device=dev)
+            o = torch.empty(T, nh, dv, device=dev)
+            ms = time_graph(lambda: gq4.mla_absorb_q(W, nh, dn, dv, qn, ql), args.reps, flush)
+            report(f"mla_absorb_q_kvb28672x512_t{T}", ms, nh * wbytes(dn, R) + qn.numel() * 2 + ql.numel() * 4, peak)
+            ms = time_graph(lambda: gq4.mla_absorb_v(W, nh, dn, dv, lat, o), args.reps, flush)
+            report(f"mla_absorb_v_kvb28672x512_t{T}", ms, nh * wbytes(dv, R) + lat.numel() * 2 + o.numel() * 4, peak)
 
 
 if __name__ == "__main__":
