@@ -8,23 +8,20 @@
 //   * q is turned into bf16 exactly (integers -8..7) by the math warps and written to
 //     shared memory in the 128-byte-swizzled K-major layout the MMA reads;
 //   * for each 64-wide group the MMA warp issues four M=128 x N x K=16 tcgen05.mma into
-//     one of three TMEM partial buffers (accumulate off for the first), then commits once
-//     to a ring of "group done" barriers that the promotion (partial ready), the dequant
-//     warps (A stage free) and the activation producer (X slot free) all wait on;
+//     one of two TMEM partial buffers (accumulate off for the first), then commits;
 //   * the math warps load the partial (tcgen05.ld), multiply it by the row's scale of
-//     that group and add it to running sums kept in registers ("promotion", packed f32x2
-//     FMAs), then free the buffer -- the MMAs of groups g+1 and g+2 overlap the promotion
-//     of group g.
+//     that group and add it to running sums kept in registers ("promotion"), then free
+//     the buffer -- the MMA of group g+1 overlaps the promotion of group g.
 // TMEM lane = weight row, so the scale is one register per thread and group.
 //
 // Warp roles (512 threads = 4 warpgroups, one CTA per SM, persistent over units):
 //   WG0  warp 0  TMA producer of the packed nibble tiles: 128 rows x 128 B (four groups,
 //                swizzle 128B) per stage in two 64-row boxes, 5-stage ring
 //        warp 1  TMEM allocation and the MMA issuer (one thread)
-//        warp 2  TMA producer of the activation tiles (N <= 160 rows x 64 bf16, swizzle
+//        warp 2  TMA producer of the activation tiles (N <= 192 rows x 64 bf16, swizzle
 //                128B) as 128/64/32/16-row boxes, 4-stage ring; warp 3 idle
 //   (TMA cost is per request more than per byte: few large boxes keep the rings fed)
-//   WG1  warps 4-7   dequant: rows [32d, 32d+32) of the bf16 A tile, 3-slot ring
+//   WG1  warps 4-7   dequant: rows [32d, 32d+32) of the bf16 A tile, 4-slot ring
 //   WG2-3 warps 8-15 promotion: TMEM lane quarter (warp % 4) x column half, running
 //                sums in registers, epilogue
 // setmaxnreg moves registers from WG0/WG1 (48 each) to the promotion warps (200 each):
@@ -46,13 +43,9 @@ constexpr int kTcThreads = 512;
 constexpr int kTcWStages = 5;                                   // packed-weight ring, 4 groups/stage
 constexpr int kTcXStages = 4;                                   // activation ring, 1 group/stage
 constexpr int kTcAStages = 3;                                   // dequantised bf16 A tiles
-constexpr int kTcPBufs = 3;                                     // TMEM partial buffers
-constexpr int kTcDone = 8;                                      // "MMAs of group g done" barrier ring
-constexpr int kTcMaxN = 160;                                    // rows per pass (TMEM, registers)
-constexpr int kTcChunks = 3;                                    // 32-column chunks 2c + half, c < 3
-static_assert(2 * kTcChunks * 32 >= kTcMaxN, "chunks cover a pass");
-static_assert(kTcPBufs * kTcMaxN <= 512, "TMEM columns");
-static_assert(kTcDone >= 2 * (kTcXStages > kTcAStages ? kTcXStages : kTcAStages), "no phase aliasing");
+constexpr int kTcMaxN = 192;                                   // rows per pass (TMEM, registers)
+constexpr int kTcChunks = kTcMaxN / 64;                         // 32-column chunks per column half
+static_assert(kTcChunks == 3, "the promotion reads chunks 2c + half, c < 3");
 constexpr int kTcWGroups = 4;                                   // groups per weight stage
 constexpr int kTcWBytes = 128 * 32 * kTcWGroups;                // 128 rows x 256 nibbles
 constexpr int kTcXBytes = kTcMaxN * 128;                        // N rows x 64 bf16
@@ -63,7 +56,7 @@ constexpr int kTcOffW = kTcOffA + kTcAStages * kTcABytes;
 constexpr int kTcOffBar = kTcOffW + kTcWStages * kTcWBytes;
 constexpr int kTcSmemBytes = kTcOffBar + 512 + 1024;            // + 1024 for alignment
 static_assert(kTcSmemBytes <= 232448, "shared memory per CTA");
-constexpr int kTcTmemCols = 512;                                // three N<=160 partials (power of 2)
+constexpr int kTcTmemCols = 512;                                // two N<=192 partials (power of 2)
 constexpr int kStatusTimeout = 8;                               // GQ4_ERR_TIMEOUT
 
 struct TcParams {
@@ -195,6 +188,20 @@ __device__ __forceinline__ uint64_t splat2(float s) {
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// The registers a tcgen05.ld writes hold their values only after tcgen05.wait::ld, but
+// the compiler sees them as written by the load itself and may move arithmetic on them
+// above the wait.  Passing them through an empty volatile asm placed after the wait
+// makes every later use depend on it.
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                   "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                   "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
 
 // ---------------------------------------------------------------- the kernel
 template <int MODE>  // 0: gate+up with SiLU(g)*u -> h (bf16); 1: down -> y += w * D
@@ -209,14 +216,15 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
     const uint32_t sb = smem_u32(smem);
     const uint32_t bar0 = sb + kTcOffBar;
     auto wfull_bar = [&](int s) { return bar0 + 8 * s; };
-    auto wempty_bar = [&](int s) { return bar0 + 64 + 8 * s; };
-    auto xfull_bar = [&](int s) { return bar0 + 128 + 8 * s; };
-    auto afull_bar = [&](int a) { return bar0 + 192 + 8 * a; };
-    auto pempty_bar = [&](int b) { return bar0 + 224 + 8 * b; };
-    auto done_bar = [&](uint32_t g) { return bar0 + 256 + 8 * (g % kTcDone); };
-    auto done_par = [](uint32_t g) { return (g / kTcDone) & 1; };
-    uint32_t *tmem_slot = (uint32_t *)(smem + kTcOffBar + 320);
-    volatile int *abort_flag = (volatile int *)(smem + kTcOffBar + 324);
+    auto wempty_bar = [&](int s) { return bar0 + 96 + 8 * s; };
+    auto xfull_bar = [&](int s) { return bar0 + 192 + 8 * s; };
+    auto xempty_bar = [&](int s) { return bar0 + 232 + 8 * s; };
+    auto afull_bar = [&](int a) { return bar0 + 272 + 8 * a; };
+    auto aempty_bar = [&](int a) { return bar0 + 296 + 8 * a; };
+    auto pfull_bar = [&](int b) { return bar0 + 320 + 8 * b; };
+    auto pempty_bar = [&](int b) { return bar0 + 336 + 8 * b; };
+    uint32_t *tmem_slot = (uint32_t *)(smem + kTcOffBar + 360);
+    volatile int *abort_flag = (volatile int *)(smem + kTcOffBar + 368);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -224,10 +232,18 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
             mbar_init(wfull_bar(s), 1);
             mbar_init(wempty_bar(s), 4);  // the four dequant warps
         }
-        for (int s = 0; s < kTcXStages; ++s) mbar_init(xfull_bar(s), 1);
-        for (int a = 0; a < kTcAStages; ++a) mbar_init(afull_bar(a), 4);
-        for (int b = 0; b < kTcPBufs; ++b) mbar_init(pempty_bar(b), 8);
-        for (int g = 0; g < kTcDone; ++g) mbar_init(done_bar(g), 1);  // one MMA commit per group
+        for (int s = 0; s < kTcXStages; ++s) {
+            mbar_init(xfull_bar(s), 1);
+            mbar_init(xempty_bar(s), 1);  // MMA commit
+        }
+        for (int a = 0; a < kTcAStages; ++a) {
+            mbar_init(afull_bar(a), 4);
+            mbar_init(aempty_bar(a), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(pfull_bar(b), 1);
+            mbar_init(pempty_bar(b), 8);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_async_smem();
@@ -275,10 +291,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                     } else {
                         for (int G = 0; G < p.ng; ++G, ++it) {
                             const int s = it % nst;
-                            // the slot's previous tile (group it - nst) must have been consumed
-                            if (it >= (uint32_t)nst &&
-                                !(ok = mbar_wait(done_bar(it - nst), done_par(it - nst), abort_flag, p.status)))
-                                break;
+                            if (!(ok = mbar_wait(xempty_bar(s), ((it / nst) & 1) ^ 1, abort_flag, p.status))) break;
                             const uint32_t dst = sb + kTcOffX + s * kTcXBytes;
                             mbar_expect_tx(xfull_bar(s), N * 128);
                             int r = 0;  // N (a multiple of 16) as 128/64/32/16-row boxes
@@ -313,26 +326,30 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                     const int N = (min(kTcMaxN, cnt - n0) + 15) & ~15;
                     const uint32_t idesc = idesc_bf16_m128(N);
                     for (int G = 0; G < p.ng; ++G, ++it) {
-                        const int xs = it % kTcXStages, as = it % kTcAStages, b = it % kTcPBufs;
+                        const int xs = it % kTcXStages, as = it % kTcAStages, b = it & 1;
                         ok = mbar_wait(xfull_bar(xs), (it / kTcXStages) & 1, abort_flag, p.status) &&
                              mbar_wait(afull_bar(as), (it / kTcAStages) & 1, abort_flag, p.status) &&
-                             mbar_wait(pempty_bar(b), ((it / kTcPBufs) & 1) ^ 1, abort_flag, p.status);
+                             mbar_wait(pempty_bar(b), ((it >> 1) & 1) ^ 1, abort_flag, p.status);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t a_addr = sb + kTcOffA + as * kTcABytes;
                         const uint32_t x_addr = sb + kTcOffX + xs * kTcXBytes;
                         #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            tc_mma(tmem + b * kTcMaxN, sw128_desc(a_addr + kk * 32),
+                            tc_mma(tmem + b * 256, sw128_desc(a_addr + kk * 32),
                                    sw128_desc(x_addr + kk * 32), idesc, kk > 0 ? 1u : 0u);
-                        // one commit tells the promotion (partial ready), the dequant warps (A
-                        // stage free) and the activation producer (X slot free)
-                        tc_commit(done_bar(it));
+                        tc_commit(pfull_bar(b));
+                        tc_commit(aempty_bar(as));
+                        tc_commit(xempty_bar(xs));
                     }
                 }
             }
-            // the last commit must have arrived before the CTA's shared memory is released
-            if (ok && it > 0) mbar_wait(done_bar(it - 1), done_par(it - 1), abort_flag, p.status);
+            // the last commits must have arrived before the CTA's shared memory is released
+            if (ok && it > 0) {
+                const uint32_t j = it - 1;
+                mbar_wait(xempty_bar(j % kTcXStages), (j / kTcXStages) & 1, abort_flag, p.status);
+                mbar_wait(aempty_bar(j % kTcAStages), (j / kTcAStages) & 1, abort_flag, p.status);
+            }
         }
         __syncwarp();
       } else if (warp >= 4) {
@@ -357,9 +374,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                     if ((G & 3) == 0 &&
                         !(ok = mbar_wait(wfull_bar(ws), (wi / kTcWStages) & 1, abort_flag, p.status)))
                         break;
-                    // the A stage's previous tile (group it - kTcAStages) must have been consumed
-                    if (it >= (uint32_t)kTcAStages &&
-                        !(ok = mbar_wait(done_bar(it - kTcAStages), done_par(it - kTcAStages), abort_flag, p.status)))
+                    if (!(ok = mbar_wait(aempty_bar(as), ((it / kTcAStages) & 1) ^ 1, abort_flag, p.status)))
                         break;
                     // packed tile (128B-swizzled): row pr at pr*128, its 16-byte chunk c at
                     // (c ^ (pr & 7)) * 16; group G%4 is chunks 2(G%4), 2(G%4)+1; rows
@@ -400,7 +415,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
         const int lrow = 32 * q + lane;      // TMEM lane = A row
         uint32_t it = 0;
         bool ok = true;
-        float2 acc[kTcChunks][16];  // chunk c: columns 32(2c + half) + 2j, + 2j + 1
+        float acc[kTcChunks][32];
 
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
             const int a = u / p.m_tiles, mt = u - a * p.m_tiles;
@@ -418,60 +433,62 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                 #pragma unroll
                 for (int c = 0; c < kTcChunks; ++c)
                     #pragma unroll
-                    for (int j = 0; j < 16; ++j) acc[c][j] = make_float2(0.f, 0.f);
-                // chunks 2c + half of 32 columns; the first two are loaded together
-                const int col0 = 32 * half, col1 = 32 * (2 + half), col2 = 32 * (4 + half);
-                // scales four groups at a time, prefetched one float4 ahead (ng % 4 == 0);
-                // the four groups of a float4 are unrolled so each takes its scale directly
+                    for (int j = 0; j < 32; ++j) acc[c][j] = 0.f;
+                // scales four groups at a time, prefetched one float4 ahead (ng % 4 == 0)
                 float4 s_cur = *(const float4 *)srow;
                 float4 s_next = p.ng > 4 ? *(const float4 *)(srow + 4) : s_cur;
-                for (int G = 0; G < p.ng; G += 4) {
-                    #pragma unroll
-                    for (int gq = 0; gq < 4; ++gq, ++it) {
-                        const float sc = gq == 0 ? s_cur.x : gq == 1 ? s_cur.y : gq == 2 ? s_cur.z : s_cur.w;
-                        const uint32_t b = it % kTcPBufs;
-                        if (!(ok = mbar_wait(done_bar(it), done_par(it), abort_flag, p.status))) break;
-                        tc_fence_after();
-                        const float2 s2 = make_float2(sc, sc);
-                        const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + b * kTcMaxN;
-                        auto release = [&]() {  // this warp has read all it needs of buffer b
+                for (int G = 0; G < p.ng; ++G, ++it) {
+                    const int gq = G & 3;
+                    const float sc = gq == 0 ? s_cur.x : gq == 1 ? s_cur.y : gq == 2 ? s_cur.z : s_cur.w;
+                    if (gq == 3) {
+                        s_cur = s_next;
+                        if (G + 5 < p.ng) s_next = *(const float4 *)(srow + G + 5);
+                    }
+                    const int b = it & 1;
+                    if (!(ok = mbar_wait(pfull_bar(b), (it >> 1) & 1, abort_flag, p.status))) break;
+                    tc_fence_after();
+                    const uint64_t ss = splat2(sc);
+                    const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + b * 256;
+                    // chunks 2c + half of 32 columns; the first two are loaded together
+                    const int col0 = 32 * half, col1 = 32 * (2 + half), col2 = 32 * (4 + half);
+                    if (col0 < N) {
+                        uint32_t r0[32], r1[32];
+                        tmem_ld32(tbase + col0, r0);
+                        if (col1 < N) tmem_ld32(tbase + col1, r1);
+                        tmem_wait_ld();
+                        tmem_regs_ready(r0);
+                        if (col1 < N) tmem_regs_ready(r1);
+                        if (col2 >= N) {  // nothing else to read: the buffer may be reused
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(pempty_bar(b));
-                        };
-                        if (col0 < N) {
-                            uint32_t r0[32], r1[32];
-                            tmem_ld32(tbase + col0, r0);
-                            if (col1 < N) tmem_ld32(tbase + col1, r1);
-                            tmem_wait_ld();
-                            if (col2 >= N) release();
-                            #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                acc[0][j] = __ffma2_rn(make_float2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])),
-                                                       s2, acc[0][j]);
-                            if (col1 < N) {
-                                #pragma unroll
-                                for (int j = 0; j < 16; ++j)
-                                    acc[1][j] = __ffma2_rn(make_float2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1])),
-                                                           s2, acc[1][j]);
-                            }
-                        } else {
-                            release();  // a pass of <= 32 rows: this warp owns no chunk
                         }
-                        if (col2 < N) {
-                            uint32_t r2[32];
-                            tmem_ld32(tbase + col2, r2);
-                            tmem_wait_ld();
-                            release();
+                        #pragma unroll
+                        for (int j = 0; j < 32; j += 2)
+                            fma2(acc[0][j], acc[0][j + 1], __uint_as_float(r0[j]), __uint_as_float(r0[j + 1]), ss);
+                        if (col1 < N) {
                             #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                acc[2][j] = __ffma2_rn(make_float2(__uint_as_float(r2[2 * j]), __uint_as_float(r2[2 * j + 1])),
-                                                       s2, acc[2][j]);
+                            for (int j = 0; j < 32; j += 2)
+                                fma2(acc[1][j], acc[1][j + 1], __uint_as_float(r1[j]), __uint_as_float(r1[j + 1]), ss);
                         }
                     }
-                    if (!ok) break;
-                    s_cur = s_next;
-                    if (G + 8 < p.ng) s_next = *(const float4 *)(srow + G + 8);
+                    if (col2 < N) {
+                        uint32_t r2[32];
+                        tmem_ld32(tbase + col2, r2);
+                        tmem_wait_ld();
+                        tmem_regs_ready(r2);
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(pempty_bar(b));
+                        #pragma unroll
+                        for (int j = 0; j < 32; j += 2)
+                            fma2(acc[2][j], acc[2][j + 1], __uint_as_float(r2[j]), __uint_as_float(r2[j + 1]), ss);
+                    }
+                    if (half == 1 && N <= 32) {  // this warp owns no chunk of this pass
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(pempty_bar(b));
+                    }
                 }
                 if (!ok) break;
                 // ---------------------------------------------------- epilogue
@@ -484,10 +501,9 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                         if (col < N) {
                             #pragma unroll
                             for (int j = 0; j < 32; ++j) {
-                                const float av = (j & 1) ? acc[c][j >> 1].y : acc[c][j >> 1].x;
-                                const float uv = __shfl_xor_sync(0xffffffffu, av, 1);
+                                const float uv = __shfl_xor_sync(0xffffffffu, acc[c][j], 1);
                                 if (!(lane & 1) && col + j < nrows) {
-                                    const float g = av;
+                                    const float g = acc[c][j];
                                     const float hv = g / (1.0f + expf(-g)) * uv;
                                     p.h[(int64_t)(row0 + n0 + col + j) * p.O + f] = (uint16_t)bf16_bits_rn(hv);
                                 }
@@ -512,8 +528,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                             for (int j = 0; j < 32; ++j) {
                                 const int tok = __shfl_sync(0xffffffffu, tok_l, j);
                                 const float wt = __shfl_sync(0xffffffffu, wt_l, j);
-                                const float av = (j & 1) ? acc[c][j >> 1].y : acc[c][j >> 1].x;
-                                if (col + j < nrows) atomicAdd(p.y + (int64_t)tok * p.O + o, wt * av);
+                                if (col + j < nrows) atomicAdd(p.y + (int64_t)tok * p.O + o, wt * acc[c][j]);
                             }
                         }
                     }
