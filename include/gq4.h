@@ -281,7 +281,9 @@ gq4_status gq4_matvec_rows(const gq4_tensor *W, const int32_t *idx, int64_t n_se
  *      q_lat: device f32 [T][n_heads][R].
  * gq4_mla_absorb_v: o[t][h][v] = sum_{c < R} lat[t][h][c] * w(h*D + d_nope + v, c)
  *      lat: device [T][n_heads][R] of ldt; o: device f32 [T][n_heads][d_v].
- * fp32 accumulation.  T <= 262140.  Outputs must not overlap the inputs or W. */
+ * fp32 accumulation.  T <= 262140.  Outputs must not overlap the inputs or W.  The Q
+ * projection may split a head's key rows over several blocks whose sums meet through
+ * float atomics, so its last bits can differ from call to call. */
 gq4_status gq4_mla_absorb_q(const gq4_tensor *W, int32_t n_heads, int32_t d_nope, int32_t d_v,
                             const void *q_nope, gq4_dtype qdt, int64_t T, float *q_lat,
                             gq4_stream_t stream);

@@ -238,7 +238,9 @@ def _toy(T, E, K, H=128, F=128, seed=3, **kw):
                                        # TMA-fed decode kernel for gate+up and down (H, F multiples
                                        # of 256), alone and beside the tensor-core path
                                        (12, 16, 4, 256, 256), (30, 8, 8, 512, 256), (20, 64, 8, 256, 512),
-                                       (9, 4, 4, 768, 1280)])
+                                       (9, 4, 4, 768, 1280),
+                                       # few experts: 32-row gate+up bands
+                                       (1, 16, 4, 512, 1536), (2, 4, 2, 256, 512)])
 def test_moe_small_full_oracle(T, E, K, H, F):
     s = MoESet(_toy(T, E, K, H, F))
     y, ws = s.run()

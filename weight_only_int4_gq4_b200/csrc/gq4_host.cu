@@ -378,8 +378,9 @@ gq4_status launch_stream_k(const StreamMats &m, const SkinnyParams &p, int units
 
 // Band height: the tallest whose unit count gives every SM at least two bands (gate+up:
 // 128 or 64 rows of each matrix; down and plain matvec: 256, 128 or 64 rows), else the
-// smallest.  The n-tile count covers the columns of one pass.  `mats` = matrices
-// (experts) the call may touch.
+// smallest.  (32-row gate+up bands balance one token's experts better on paper but ran
+// slower: their TMA boxes and stages are too small to keep HBM busy.)  The n-tile count
+// covers the columns of one pass.  `mats` = matrices (experts) the call may touch.
 template <int MODE, int NT>
 gq4_status launch_stream_nt(const StreamMats &m, const SkinnyParams &p, int mats, int32_t *status,
                             cudaStream_t st) {
@@ -1068,8 +1069,14 @@ extern "C" gq4_status gq4_mla_absorb_q(const gq4_tensor *W, int32_t n_heads, int
     const int nsplit = words >= kMlaThreads ? 1 : kMlaThreads / words;
     const int threads = words >= kMlaThreads ? kMlaThreads : words * nsplit;
     const size_t smem = ((size_t)kMlaTok * d_nope + (nsplit > 1 ? (size_t)nsplit * kMlaTok * R : 0)) * 4;
-    const dim3 grid((unsigned)n_heads, (unsigned)((T + kMlaTok - 1) / kMlaTok));
+    // key rows of a head split over blockIdx.z until the grid covers about two waves of
+    // SMs (at least 16 rows per slice); the slices add into a zeroed output
+    const int64_t tblocks = (T + kMlaTok - 1) / kMlaTok;
+    int zs = (int)std::max<int64_t>(1, (2 * sm_count()) / ((int64_t)n_heads * tblocks));
+    zs = std::max(1, std::min(zs, d_nope / 16));
+    const dim3 grid((unsigned)n_heads, (unsigned)tblocks, (unsigned)zs);
     cudaStream_t s = S(stream);
+    if (zs > 1 && cudaMemsetAsync(q_lat, 0, (size_t)T * n_heads * R * 4, s) != cudaSuccess) return GQ4_ERR_CUDA;
     if (qdt == GQ4_F32)
         gq4_mla_q_kernel<0><<<grid, threads, smem, s>>>((const uint32_t *)W->w, W->s, R, W->ng, W->gs, n_heads,
                                                         d_nope, d_v, q_nope, T, q_lat);

@@ -31,11 +31,14 @@ __device__ __forceinline__ float mla_act(const void *x, int64_t i) {
     return __uint_as_float((uint32_t)((const uint16_t *)x)[i] << 16);
 }
 
-// Q absorb.  Block: one head and kMlaTok tokens.  With W = R/8 packed words per row, the
-// block has W x nsplit threads (nsplit = 256 / W when W <= 256, else 256 threads over
-// the words in turn): thread (split, j) owns columns 8j..8j+7 (one device word, all in
-// one group since gs % 8 == 0) and sums the key rows d = split, split + nsplit, ...; the
-// splits' partial sums are added in shared memory in split order (deterministic).
+// Q absorb.  Block: one head, kMlaTok tokens and one slice of the head's key rows
+// (blockIdx.z of gridDim.z slices; with more than one slice the block adds its partial
+// sums into the zeroed output with atomics, in no fixed order).  With W = R/8 packed words
+// per row, the block has W x nsplit threads (nsplit = 256 / W when W <= 256, else 256
+// threads over the words in turn): thread (split, j) owns columns 8j..8j+7 (one device
+// word, all in one group since gs % 8 == 0) and sums the slice's key rows d = d0 + split,
+// d0 + split + nsplit, ...; the splits' partial sums are added in shared memory in split
+// order.
 template <int XDT>
 __global__ void __launch_bounds__(kMlaThreads) gq4_mla_q_kernel(const uint32_t *__restrict__ w,
                                                               const float *__restrict__ s, int R, int ng,
@@ -50,6 +53,9 @@ __global__ void __launch_bounds__(kMlaThreads) gq4_mla_q_kernel(const uint32_t *
     const bool wide = W >= (int)blockDim.x;
     const int nsplit = wide ? 1 : (int)blockDim.x / W;
     const int split = wide ? 0 : (int)threadIdx.x / W;
+    const int dper = (dn + gridDim.z - 1) / gridDim.z;
+    const int d0 = blockIdx.z * dper, d1 = min(dn, d0 + dper);
+    const bool atomic_out = gridDim.z > 1;
     float *qs = mla_sm;                 // [kMlaTok][dn]
     float *red = mla_sm + kMlaTok * dn; // [nsplit][kMlaTok][R] (nsplit > 1)
     for (int i = threadIdx.x; i < kMlaTok * dn; i += blockDim.x) {
@@ -67,7 +73,7 @@ __global__ void __launch_bounds__(kMlaThreads) gq4_mla_q_kernel(const uint32_t *
             for (int m = 0; m < 8; ++m) acc[t][m] = 0.f;
         const int g = (8 * j) / gs;
         #pragma unroll 4
-        for (int d = split; d < dn; d += nsplit) {
+        for (int d = d0 + split; d < d1; d += nsplit) {
             const int64_t row = (int64_t)h * D + d;
             const uint32_t v = __ldg(w + row * W + j);
             const float sc = __ldg(s + row * ng + g);
@@ -85,9 +91,14 @@ __global__ void __launch_bounds__(kMlaThreads) gq4_mla_q_kernel(const uint32_t *
             #pragma unroll
             for (int t = 0; t < kMlaTok; ++t) {
                 if (t >= nt) break;
-                float4 *o = (float4 *)(out + ((t0 + t) * nh + h) * (int64_t)R + 8 * j);
-                o[0] = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
-                o[1] = make_float4(acc[t][4], acc[t][5], acc[t][6], acc[t][7]);
+                float *o = out + ((t0 + t) * nh + h) * (int64_t)R + 8 * j;
+                if (atomic_out) {
+                    #pragma unroll
+                    for (int m = 0; m < 8; ++m) atomicAdd(o + m, acc[t][m]);
+                } else {
+                    ((float4 *)o)[0] = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+                    ((float4 *)o)[1] = make_float4(acc[t][4], acc[t][5], acc[t][6], acc[t][7]);
+                }
             }
         } else {
             #pragma unroll
@@ -104,15 +115,17 @@ __global__ void __launch_bounds__(kMlaThreads) gq4_mla_q_kernel(const uint32_t *
             const int t = i / R, c = i - t * R;
             float sum = 0.f;
             for (int sp = 0; sp < nsplit; ++sp) sum += red[((int64_t)sp * kMlaTok + t) * R + c];
-            out[((t0 + t) * nh + h) * (int64_t)R + c] = sum;
+            float *o = out + ((t0 + t) * nh + h) * (int64_t)R + c;
+            if (atomic_out) atomicAdd(o, sum); else *o = sum;
         }
     }
 }
 
 // V absorb.  Block: one head, kMlaTok tokens (blockIdx.z) and 8 warps of kMlaVRowsPerWarp
-// value rows each (blockIdx.y).  A warp's lanes take the row's words j = lane, lane+32,
-// ... (coalesced), form each word's partial against the staged latent values, scale it
-// by the word's group scale, and the lanes' sums meet in a shuffle reduction.
+// value rows each (blockIdx.y).  A warp's lanes take the words j = lane, lane+32, ... of
+// all its rows at once (coalesced), form each word's partial against the staged latent
+// values, scale it by the word's group scale, and the lanes' sums meet in a shuffle
+// reduction per row and token.
 template <int XDT>
 __global__ void __launch_bounds__(kMlaThreads) gq4_mla_v_kernel(const uint32_t *__restrict__ w,
                                                               const float *__restrict__ s, int R, int ng,
@@ -132,41 +145,57 @@ __global__ void __launch_bounds__(kMlaThreads) gq4_mla_v_kernel(const uint32_t *
     const int W = R >> 3;
     const int64_t D = dn + dv;
     const int v0 = (blockIdx.y * (kMlaThreads / 32) + warp) * kMlaVRowsPerWarp;
-    for (int v = v0; v < min(dv, v0 + kMlaVRowsPerWarp); ++v) {
-        const int64_t row = (int64_t)h * D + dn + v;
-        float acc[kMlaTok];
+    const int nv = min(kMlaVRowsPerWarp, dv - v0);  // rows of this warp (may be <= 0)
+    // the warp's rows are walked together so their loads are in flight at the same time
+    float acc[kMlaVRowsPerWarp][kMlaTok];
+    #pragma unroll
+    for (int r = 0; r < kMlaVRowsPerWarp; ++r)
         #pragma unroll
-        for (int t = 0; t < kMlaTok; ++t) acc[t] = 0.f;
-        for (int j = lane; j < W; j += 32) {
-            const uint32_t word = __ldg(w + row * W + j);
-            const float sc = __ldg(s + row * ng + (8 * j) / gs);
-            float qv[8];
+        for (int t = 0; t < kMlaTok; ++t) acc[r][t] = 0.f;
+    for (int j = lane; j < W && nv > 0; j += 32) {
+        uint32_t word[kMlaVRowsPerWarp];
+        float sc[kMlaVRowsPerWarp];
+        #pragma unroll
+        for (int r = 0; r < kMlaVRowsPerWarp; ++r) {
+            const int64_t row = (int64_t)h * D + dn + v0 + min(r, nv - 1);
+            word[r] = __ldg(w + row * W + j);
+            sc[r] = __ldg(s + row * ng + (8 * j) / gs);
+        }
+        float qv[kMlaVRowsPerWarp][8];  // the words decoded once, used by every token
+        #pragma unroll
+        for (int r = 0; r < kMlaVRowsPerWarp; ++r)
             #pragma unroll
-            for (int m = 0; m < 8; ++m) qv[m] = (float)dev_q(word, dev_slot(m));
+            for (int m = 0; m < 8; ++m) qv[r][m] = (float)dev_q(word[r], dev_slot(m));
+        #pragma unroll
+        for (int t = 0; t < kMlaTok; ++t) {
+            const float4 a = *(const float4 *)(mla_sm + t * R + 8 * j);
+            const float4 b = *(const float4 *)(mla_sm + t * R + 8 * j + 4);
             #pragma unroll
-            for (int t = 0; t < kMlaTok; ++t) {
-                const float4 a = *(const float4 *)(mla_sm + t * R + 8 * j);
-                const float4 b = *(const float4 *)(mla_sm + t * R + 8 * j + 4);
-                float part = qv[0] * a.x;
-                part = fmaf(qv[1], a.y, part);
-                part = fmaf(qv[2], a.z, part);
-                part = fmaf(qv[3], a.w, part);
-                part = fmaf(qv[4], b.x, part);
-                part = fmaf(qv[5], b.y, part);
-                part = fmaf(qv[6], b.z, part);
-                part = fmaf(qv[7], b.w, part);
-                acc[t] = fmaf(sc, part, acc[t]);
+            for (int r = 0; r < kMlaVRowsPerWarp; ++r) {
+                float part = qv[r][0] * a.x;
+                part = fmaf(qv[r][1], a.y, part);
+                part = fmaf(qv[r][2], a.z, part);
+                part = fmaf(qv[r][3], a.w, part);
+                part = fmaf(qv[r][4], b.x, part);
+                part = fmaf(qv[r][5], b.y, part);
+                part = fmaf(qv[r][6], b.z, part);
+                part = fmaf(qv[r][7], b.w, part);
+                acc[r][t] = fmaf(sc[r], part, acc[r][t]);
             }
         }
+    }
+    #pragma unroll
+    for (int r = 0; r < kMlaVRowsPerWarp; ++r)
         #pragma unroll
         for (int t = 0; t < kMlaTok; ++t)
             #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-        if (lane == 0) {
+            for (int off = 16; off > 0; off >>= 1) acc[r][t] += __shfl_xor_sync(0xffffffffu, acc[r][t], off);
+    if (lane == 0) {
+        #pragma unroll
+        for (int r = 0; r < kMlaVRowsPerWarp; ++r)
             #pragma unroll
             for (int t = 0; t < kMlaTok; ++t)
-                if (t < nt) out[((t0 + t) * nh + h) * (int64_t)dv + v] = acc[t];
-        }
+                if (r < nv && t < nt) out[((t0 + t) * nh + h) * (int64_t)dv + v0 + r] = acc[r][t];
     }
 }
 
