@@ -299,32 +299,48 @@ def main():
     cnt = ws.routing()["cnt"].cpu().numpy()[:cfg.E]
     split = split_experts(cfg, cnt)
 
-    # ---- device-timed steps: one moe_expert_ffn call (with its stage events) captured in
-    # a CUDA graph and replayed, so the step's kernels run without host launch gaps; L2
-    # flushed between steps, outside the events
+    # ---- device-timed steps: one moe_expert_ffn call captured in a CUDA graph and
+    # replayed, so the step's kernels run without host launch gaps, timed by events on the
+    # launching stream around the replay; L2 flushed between steps, outside the events.
+    # The stage split comes from a second graph of the same call with its stage events
+    # (event nodes inside a graph cost a few microseconds each, so they stay out of the
+    # timed step).
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(NEV)]
     for e in ev:  # torch creates the CUDA event lazily, at its first record
         e.record(stream)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
+        step()
+    graph_st = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_st):
         step(ev)
     for _ in range(args.warmup):
         graph.replay()
+        graph_st.replay()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    stage = np.zeros((args.steps, NEV - 1))
+    step_ms = np.zeros(args.steps)
+    ta, tb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
+            ta.record(stream)
             graph.replay()
-            torch.cuda.synchronize()
-            stage[i] = [ev[j].elapsed_time(ev[j + 1]) for j in range(NEV - 1)]
+            tb.record(stream)
+            tb.synchronize()
+            step_ms[i] = ta.elapsed_time(tb)
     if world > 1:
         dist.barrier()
-    step_ms = stage.sum(1)
     ms = float(step_ms.mean())
+    stage = np.zeros((args.steps, NEV - 1))
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        graph_st.replay()
+        torch.cuda.synchronize()
+        stage[i] = [ev[j].elapsed_time(ev[j + 1]) for j in range(NEV - 1)]
+    del graph, graph_st
 
     # ---- end to end through the public API, host buffers (pinned), copies timed
     x_pin = torch.from_numpy(x_h.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -387,7 +403,9 @@ def main():
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "F": cfg.F, "K": cfg.K,
                        "gs": 64, "distinct_experts": n_active, "experts_tensor_core": split["n_large"],
                        "parallelism": f"replicas x{world}",
-                       "launch": "value: CUDA-graph replay of one moe_expert_ffn call; e2e: direct calls",
+                       "launch": "value: CUDA-graph replay of one moe_expert_ffn call, events around the "
+                                 "replay; stage_ms: a second graph with the call's stage events; "
+                                 "e2e: direct calls",
                        "l2": f"{L2_FLUSH_BYTES >> 20} MiB flush between steps; touched weights "
                              f"{n_active * per_expert / 1e9:.2f} GB/step"},
             "hbm_gbs_step": step_bytes / (ms * 1e-3) / 1e9,
