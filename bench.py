@@ -136,9 +136,35 @@ def cpu_baseline(cfg: synth.MoEConfig, budget_s: float = 12.0, max_tokens: int =
         done += 1
         if elapsed >= budget_s:
             break
+    # one token on a single thread as well (the oracle's loops are otherwise spread over
+    # all host cores with OpenMP)
+    t = int(order[0])
+    need = [int(e) for e in idx[t]]
+    pg = np.stack([experts[e][0][0] for e in need]); sg = np.stack([experts[e][0][1] for e in need])
+    pu = np.stack([experts[e][1][0] for e in need]); su = np.stack([experts[e][1][1] for e in need])
+    pd = np.stack([experts[e][2][0] for e in need]); sd = np.stack([experts[e][2][1] for e in need])
+    idx_l = np.zeros_like(idx)
+    idx_l[t] = np.arange(len(need))
+    prev = oracle.set_threads(1)
+    t0 = time.perf_counter()
+    oracle.moe_tokens(pg, sg, pu, su, pd, sd, cfg.H, cfg.F, x, idx_l, wts, np.array([t]))
+    single = time.perf_counter() - t0
+    oracle.set_threads(prev)
     return {"value": done / elapsed, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{done} token(s) of {cfg.name}, whole layer per token (K={cfg.K} experts), "
-                      f"{elapsed:.1f} s, fp64 plain C"}
+                      f"{elapsed:.1f} s, fp64 plain C",
+            "single_thread_tokens_per_s": 1.0 / single, "cpu_model": cpu_model()}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def per_matrix_bytes(O, I):
@@ -398,7 +424,8 @@ def main():
         line = {
             "metric": "expert-FFN tokens/s (MoE layer, 1 B200)", "value": job_tokens_per_s(world, cfg.T, ms),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": ms, "ms_p10_p50_p90": [float(v) for v in np.percentile(step_ms, [10, 50, 90])],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "F": cfg.F, "K": cfg.K,
                        "gs": 64, "distinct_experts": n_active, "experts_tensor_core": split["n_large"],

@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.orc_mla_absorb_q.restype = None
         L.orc_mla_absorb_v.argtypes = [P, P, I64, I64, I64, I64, I64, P, I, I64, P, P]
         L.orc_mla_absorb_v.restype = None
+        L.orc_set_threads.argtypes = [I]
+        L.orc_set_threads.restype = I
         L.orc_matvec_rows.restype = None
     return _lib
 
@@ -329,3 +331,8 @@ def mla_absorb_v(packed, scales, R, nh, dn, dv, lat, gs: int = 64):
     """o [T][nh][dv] fp64 = sum_c lat[t][h][c] * w(h*(dn+dv)+dn+v, c), and its bound.
     lat [T][nh][R] f32 or bf16 bits (uint16)."""
     return _mla("v", packed, scales, R, nh, dn, dv, lat, R, gs)
+
+
+def set_threads(n: int) -> int:
+    """Threads of the oracle's OpenMP loops; returns the previous count."""
+    return lib().orc_set_threads(int(n))

@@ -28,6 +28,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_OK 0
 #define ORC_ERR_SHAPE 3
@@ -512,4 +515,19 @@ void orc_mla_absorb_v(const uint8_t *packed, const float *scales, int64_t R, int
             if (bound) bound[th * dv + v] = l1 * xmax;
         }
     }
+}
+
+/* Threads the OpenMP loops above may use (test and baseline infrastructure: the CPU
+ * baseline reports an all-core and a single-thread figure).  Returns the previous count
+ * (1 when the oracle was built without OpenMP). */
+int orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    int prev = omp_get_max_threads();
+    if (n > 0) omp_set_num_threads(n);
+    return prev;
+#else
+    (void)n;
+    return 1;
+#endif
 }
