@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define GQ4_ABI_VERSION 3u
+#define GQ4_ABI_VERSION 4u
 
 typedef struct CUstream_st *gq4_stream_t; /* binary-compatible with cudaStream_t */
 typedef struct CUevent_st *gq4_event_t;   /* binary-compatible with cudaEvent_t */
@@ -56,7 +56,7 @@ typedef enum {
     GQ4_ERR_ALIAS = 5,       /* an output overlaps an input */
     GQ4_ERR_WORKSPACE = 6,   /* workspace too small */
     GQ4_ERR_CUDA = 7,        /* a CUDA runtime call failed */
-    GQ4_ERR_TIMEOUT = 8,     /* reserved: a bounded device wait gave up */
+    GQ4_ERR_TIMEOUT = 8,     /* a bounded device wait gave up (see gq4_selftest_wait_timeout) */
     GQ4_ERR_NONFINITE_LOGIT = 9 /* a router row held NaN/+inf, or no finite maximum */
 } gq4_status;
 
@@ -290,6 +290,17 @@ gq4_status gq4_mla_absorb_q(const gq4_tensor *W, int32_t n_heads, int32_t d_nope
 gq4_status gq4_mla_absorb_v(const gq4_tensor *W, int32_t n_heads, int32_t d_nope, int32_t d_v,
                             const void *lat, gq4_dtype ldt, int64_t T, float *o,
                             gq4_stream_t stream);
+
+/* ---- self-test of the bounded device wait
+ * Every wait of the library's kernels (on an mbarrier that a TMA copy, a tensor-core
+ * commit or another warp completes) gives up after a time limit (2 s in the kernels),
+ * raises GQ4_ERR_TIMEOUT in the call's status word and lets the kernel end, so a stuck
+ * producer never hangs the GPU.  This call runs that wait on a barrier nothing arrives
+ * on, with a limit of limit_us microseconds (1 .. 1,000,000), so that the path can be
+ * tested without a fault.
+ *   status: 16-byte aligned device int32, OR-ed with GQ4_ERR_TIMEOUT when the wait
+ *   gives up (the caller clears it first).  Asynchronous on `stream`. */
+gq4_status gq4_selftest_wait_timeout(uint32_t limit_us, int32_t *status, gq4_stream_t stream);
 
 /* moe_expert_ffn_noalloc: the same layer as moe_expert_ffn, for callers that cannot
  * allocate device memory -- a plug-in whose host program owns every device allocation

@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = gq4.lib()
-    assert lib.gq4_abi_version() == 3
+    assert lib.gq4_abi_version() == 4
     for st in range(10):
         assert lib.gq4_status_string(st).decode()
     assert lib.gq4_status_string(77) == b"unknown status"
@@ -206,3 +206,12 @@ def test_mla_absorb_argument_checks():
         assert c(out=0x700000) == gq4.ERR_ALIAS
     big = _desc(out=1025 + 7, in_=64)
     assert L.gq4_mla_absorb_q(ctypes.byref(big), 1, 1025, 7, 0x700000, 0, 1, 0x900000, None) == gq4.ERR_UNSUPPORTED
+
+
+def test_wait_selftest_argument_checks():
+    """The wait self-test refuses bad arguments before launching (fake pointers)."""
+    L = gq4.lib()
+    assert L.gq4_selftest_wait_timeout(1000, None, None) == gq4.ERR_NULL
+    assert L.gq4_selftest_wait_timeout(1000, 0x100004, None) == gq4.ERR_ALIGN
+    assert L.gq4_selftest_wait_timeout(0, 0x100000, None) == gq4.ERR_SHAPE
+    assert L.gq4_selftest_wait_timeout(2000000, 0x100000, None) == gq4.ERR_SHAPE

@@ -1115,3 +1115,14 @@ extern "C" gq4_status gq4_mla_absorb_v(const gq4_tensor *W, int32_t n_heads, int
                                                             n_heads, d_nope, d_v, lat, T, o);
     return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------------------
+// Self-test of the bounded device wait
+// ---------------------------------------------------------------------------------------
+extern "C" gq4_status gq4_selftest_wait_timeout(uint32_t limit_us, int32_t *status, gq4_stream_t stream) {
+    if (!status) return GQ4_ERR_NULL;
+    if (!aligned16(status)) return GQ4_ERR_ALIGN;
+    if (limit_us < 1 || limit_us > 1000000) return GQ4_ERR_SHAPE;
+    gq4_wait_selftest_kernel<<<1, 32, 0, S(stream)>>>(status, (uint64_t)limit_us * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
+}

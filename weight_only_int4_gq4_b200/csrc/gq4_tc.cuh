@@ -110,21 +110,40 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 // Wait for the phase of `parity` to complete; false if the CTA aborted or ~2 s passed.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          int32_t *status) {
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                              int32_t *status, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait_sleep(bar, parity)) return true;
         if ((i & 7) == 0) {
             if (*abort_flag) return false;
-            if (global_ns() - t0 > 2000000000ull) {
+            if (global_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 atomicOr(status, kStatusTimeout);
                 return false;
             }
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status) {
+    return mbar_wait_for(bar, parity, abort_flag, status, 2000000000ull);
+}
+
+// Self-test of the bounded wait every kernel uses: one thread waits on an mbarrier that
+// nothing arrives on, with a short limit; the wait gives up, raises GQ4_ERR_TIMEOUT in
+// the status word and returns, and the kernel ends normally (no trap, no hang).
+__global__ void gq4_wait_selftest_kernel(int32_t *status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_for(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint32_t bar) {

@@ -16,7 +16,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgq4.so")
-ABI_VERSION = 3
+ABI_VERSION = 4
 MOE_STAGE_EVENTS = 6
 MOE_LARGE_MIN_ROWS = 33  # GQ4_MOE_LARGE_MIN_ROWS
 NOALLOC_SCRATCH_BYTES = 16 << 20  # GQ4_NOALLOC_SCRATCH_BYTES
@@ -74,6 +74,7 @@ _SIGS = {
     "gq4_matvec_rows": ([_TP, _P, _I64, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
     "gq4_mla_absorb_q": ([_TP, _I32, _I32, _I32, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
     "gq4_mla_absorb_v": ([_TP, _I32, _I32, _I32, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
+    "gq4_selftest_wait_timeout": ([ctypes.c_uint32, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -415,3 +416,11 @@ def mla_absorb_v(W: Tensor, n_heads: int, d_nope: int, d_v: int, lat: torch.Tens
     _check(_lib.gq4_mla_absorb_v(W.ref(), n_heads, d_nope, d_v, lat.data_ptr(), _xdt(lat), T,
                                  o.data_ptr(), _stream(stream)), "gq4_mla_absorb_v")
     return o
+
+
+def selftest_wait_timeout(limit_us: int = 1000, stream=None) -> int:
+    """Runs the kernels' bounded wait on a barrier nothing completes; returns the status
+    word it leaves (GQ4_ERR_TIMEOUT when the wait gave up as designed)."""
+    st = torch.zeros(4, dtype=torch.int32, device="cuda")
+    _check(_lib.gq4_selftest_wait_timeout(limit_us, st.data_ptr(), _stream(stream)), "gq4_selftest_wait_timeout")
+    return int(st[0].item())
