@@ -33,11 +33,18 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources' code (comments and blank space left out), tying a
+    stored traffic figure to the code it was measured on."""
+    import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "weight_only_int4_gq4_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            code = fh.read()
+        code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
+        code = re.sub(r"//[^\n]*", " ", code)
+        code = " ".join(code.split())
+        h.update(f.encode() + code.encode())
     return h.hexdigest()[:16]
 
 

@@ -21,7 +21,7 @@
 //        warp 2  TMA producer of the activation tiles (N <= 192 rows x 64 bf16, swizzle
 //                128B) as 128/64/32/16-row boxes, 4-stage ring; warp 3 idle
 //   (TMA cost is per request more than per byte: few large boxes keep the rings fed)
-//   WG1  warps 4-7   dequant: rows [32d, 32d+32) of the bf16 A tile, 4-slot ring
+//   WG1  warps 4-7   dequant: rows [32d, 32d+32) of the bf16 A tile, 3-slot ring
 //   WG2-3 warps 8-15 promotion: TMEM lane quarter (warp % 4) x column half, running
 //                sums in registers, epilogue
 // setmaxnreg moves registers from WG0/WG1 (48 each) to the promotion warps (200 each):
