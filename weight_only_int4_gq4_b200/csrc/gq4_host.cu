@@ -372,7 +372,23 @@ gq4_status launch_stream_k(const StreamMats &m, const SkinnyParams &p, int units
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return GQ4_ERR_CUDA;
     const int grid = std::max(1, std::min(units_upper, sm_count()));
-    kern<<<grid, kStThreads, smem, st>>>(tm[0], tm[1], tm[2], tm[3], p, a);
+    if constexpr (ModeTraits<MODE>::kMoe) {
+        // programmatic dependent launch: the kernel may start while the one ahead of it
+        // finishes, and waits for that kernel's results inside (griddepcontrol.wait)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(kStThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, tm[0], tm[1], tm[2], tm[3], p, a) != cudaSuccess) return GQ4_ERR_CUDA;
+    } else {
+        kern<<<grid, kStThreads, smem, st>>>(tm[0], tm[1], tm[2], tm[3], p, a);
+    }
     return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
 }
 

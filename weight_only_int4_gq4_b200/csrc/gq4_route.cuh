@@ -262,6 +262,9 @@ __global__ void __launch_bounds__(1024) gq4_route_rowmap_small_kernel(
     int32_t *wcnt = sm_dyn + E;    // [32][E]
     __shared__ int sh[32];
     const int warp = threadIdx.x >> 5;
+    // the expert kernels after this one may start their prologues now; they wait for
+    // this kernel's results (griddepcontrol.wait) before reading them
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x < 4) status[threadIdx.x] = 0;
     __syncthreads();
     for (int t = warp; t < T; t += 32)

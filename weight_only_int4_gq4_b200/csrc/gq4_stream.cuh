@@ -184,6 +184,14 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
              i += (int64_t)gridDim.x * blockDim.x)
             z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    if constexpr (TR::kMoe) {
+        // MoE launches may start before the kernel ahead of them in the stream has
+        // finished (programmatic dependent launch): the prologue above touches nothing that
+        // kernel writes; everything below reads its results, so wait for it here
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        // and let the next MoE kernel start its own prologue
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
     __syncthreads();
 
     const int bands = (p.O + BR - 1) / BR;
