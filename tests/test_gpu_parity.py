@@ -286,12 +286,27 @@ def test_moe_batched_decode_full_size():
 
 def test_moe_prefill_full_size():
     """4096 tokens over all 256 experts; routing and the row map in full, the output
-    on 4 tokens of the seeded 256-token sample."""
+    on 32 tokens of the seeded 256-token sample (a wrong h row of any expert shows up
+    in the tokens routed to it, so the sample is wide enough to catch a fault in a
+    fraction of the tensor-core tiles)."""
     s = MoESet(synth.MOE_PREFILL)
     y, ws = s.run()
     assert ws.status() == 0
-    tokens = synth.MOE_PREFILL.sample_tokens()[::64]
+    tokens = synth.MOE_PREFILL.sample_tokens()[::8]
     s.check(y, ws, tokens)
+    del s
+    torch.cuda.empty_cache()
+
+
+def test_moe_prefill_512_tokens_32_experts():
+    """The 512-token prefill profiling case (the full-size rows per expert on 32
+    experts), checked on 64 tokens; a second call must agree with the first."""
+    s = MoESet(synth.MOE_PREFILL_E32)
+    y, ws = s.run()
+    assert ws.status() == 0
+    y2, _ = s.run()
+    assert np.allclose(y, y2, rtol=1e-5, atol=1e-4)
+    s.check(y, ws, synth.MOE_PREFILL_E32.sample_tokens())
     del s
     torch.cuda.empty_cache()
 
