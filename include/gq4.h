@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define GQ4_ABI_VERSION 4u
+#define GQ4_ABI_VERSION 5u
 
 typedef struct CUstream_st *gq4_stream_t; /* binary-compatible with cudaStream_t */
 typedef struct CUevent_st *gq4_event_t;   /* binary-compatible with cudaEvent_t */
@@ -290,6 +290,16 @@ gq4_status gq4_mla_absorb_q(const gq4_tensor *W, int32_t n_heads, int32_t d_nope
 gq4_status gq4_mla_absorb_v(const gq4_tensor *W, int32_t n_heads, int32_t d_nope, int32_t d_v,
                             const void *lat, gq4_dtype ldt, int64_t T, float *o,
                             gq4_stream_t stream);
+
+/* gq4_sync_status: waits for `stream` and reads a device status word written by the
+ * library's kernels -- the status output of gq4_route / gq4_rowmap, the status word of
+ * gq4_selftest_wait_timeout or of moe_expert_ffn_noalloc -- into *status_host (0, or the
+ * OR of GQ4_ERR_NONFINITE_LOGIT, GQ4_ERR_TIMEOUT, ... the kernels raised).  Synchronous:
+ * it returns after all work queued on `stream` before it has finished.
+ *   status_dev: 16-byte aligned device int32; status_host: host int32.
+ *   Returns GQ4_ERR_CUDA when the copy or the synchronisation fails (for example after an
+ *   earlier launch failed on the stream). */
+gq4_status gq4_sync_status(const int32_t *status_dev, gq4_stream_t stream, int32_t *status_host);
 
 /* ---- self-test of the bounded device wait
  * Every wait of the library's kernels (on an mbarrier that a TMA copy, a tensor-core

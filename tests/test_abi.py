@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = gq4.lib()
-    assert lib.gq4_abi_version() == 4
+    assert lib.gq4_abi_version() == 5
     for st in range(10):
         assert lib.gq4_status_string(st).decode()
     assert lib.gq4_status_string(77) == b"unknown status"
@@ -215,3 +215,13 @@ def test_wait_selftest_argument_checks():
     assert L.gq4_selftest_wait_timeout(1000, 0x100004, None) == gq4.ERR_ALIGN
     assert L.gq4_selftest_wait_timeout(0, 0x100000, None) == gq4.ERR_SHAPE
     assert L.gq4_selftest_wait_timeout(2000000, 0x100000, None) == gq4.ERR_SHAPE
+
+
+def test_sync_status_argument_checks():
+    """gq4_sync_status refuses null or misaligned pointers before any CUDA call."""
+    L = gq4.lib()
+    v = ctypes.c_int32(-1)
+    assert L.gq4_sync_status(None, None, ctypes.byref(v)) == gq4.ERR_NULL
+    assert L.gq4_sync_status(0x100000, None, None) == gq4.ERR_NULL
+    assert L.gq4_sync_status(0x100004, None, ctypes.byref(v)) == gq4.ERR_ALIGN
+    assert v.value == -1

@@ -110,3 +110,14 @@ def test_bounded_wait_gives_up_and_the_context_survives():
     y = gq4.matvec(W, bf16_to_torch(xh)).cpu().numpy()
     y_o, b = oracle.matvec(p, s, xh)
     check_close(y, y_o, b, "matvec after the wait self-test")
+
+
+def test_sync_status_reads_the_router_status_word():
+    """A router row with a NaN logit raises GQ4_ERR_NONFINITE_LOGIT in the status word;
+    gq4_sync_status waits for the stream and reads it."""
+    lg = torch.randn(3, 16, device="cuda")
+    lg[1, 4] = float("nan")
+    _, _, st = gq4.route(lg, 2)
+    assert gq4.sync_status(st) == gq4.ERR_NONFINITE_LOGIT
+    _, _, st = gq4.route(torch.randn(3, 16, device="cuda"), 2)
+    assert gq4.sync_status(st) == 0

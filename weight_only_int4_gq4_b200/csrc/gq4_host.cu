@@ -1142,3 +1142,16 @@ extern "C" gq4_status gq4_selftest_wait_timeout(uint32_t limit_us, int32_t *stat
     gq4_wait_selftest_kernel<<<1, 32, 0, S(stream)>>>(status, (uint64_t)limit_us * 1000ull);
     return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------------------
+// Reading a device status word
+// ---------------------------------------------------------------------------------------
+extern "C" gq4_status gq4_sync_status(const int32_t *status_dev, gq4_stream_t stream, int32_t *status_host) {
+    if (!status_dev || !status_host) return GQ4_ERR_NULL;
+    if (!aligned16(status_dev)) return GQ4_ERR_ALIGN;
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, status_dev, 4, cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess) return GQ4_ERR_CUDA;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return GQ4_ERR_CUDA;
+    *status_host = v;
+    return GQ4_OK;
+}

@@ -16,7 +16,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgq4.so")
-ABI_VERSION = 4
+ABI_VERSION = 5
 MOE_STAGE_EVENTS = 6
 MOE_LARGE_MIN_ROWS = 33  # GQ4_MOE_LARGE_MIN_ROWS
 NOALLOC_SCRATCH_BYTES = 16 << 20  # GQ4_NOALLOC_SCRATCH_BYTES
@@ -75,6 +75,7 @@ _SIGS = {
     "gq4_mla_absorb_q": ([_TP, _I32, _I32, _I32, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
     "gq4_mla_absorb_v": ([_TP, _I32, _I32, _I32, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
     "gq4_selftest_wait_timeout": ([ctypes.c_uint32, _P, _P], ctypes.c_int),
+    "gq4_sync_status": ([_P, _P, ctypes.POINTER(_I32)], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -423,4 +424,12 @@ def selftest_wait_timeout(limit_us: int = 1000, stream=None) -> int:
     word it leaves (GQ4_ERR_TIMEOUT when the wait gave up as designed)."""
     st = torch.zeros(4, dtype=torch.int32, device="cuda")
     _check(_lib.gq4_selftest_wait_timeout(limit_us, st.data_ptr(), _stream(stream)), "gq4_selftest_wait_timeout")
-    return int(st[0].item())
+    return sync_status(st, stream)
+
+
+def sync_status(status: torch.Tensor, stream=None) -> int:
+    """Waits for the stream and returns the device status word status[0]."""
+    _need_cuda(status)
+    v = _I32()
+    _check(_lib.gq4_sync_status(status.data_ptr(), _stream(stream), ctypes.byref(v)), "gq4_sync_status")
+    return v.value
