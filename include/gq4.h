@@ -164,7 +164,9 @@ gq4_status gq4_route(const float *logits, int64_t T, int32_t E, int32_t K, int32
  * "Device-side MoE row map": histogram, scan and fill with no host round trip).
  * Rows of an expert are ordered by ascending flat slot f = t*K + j.  Writes cnt [E],
  * offs [E+1], row_tok / row_slot / slot_row [T*K], n_active [1], active [E] (device).
- * `scratch` is device memory of gq4_rowmap_scratch_bytes(T, K, E) bytes. */
+ * `scratch` is device memory of gq4_rowmap_scratch_bytes(T, K, E) bytes; its first
+ * int32 is the call's status word: GQ4_ERR_SHAPE is OR-ed in when an idx entry lies
+ * outside [0, E), and the tables are then not valid (read it with gq4_sync_status). */
 size_t gq4_rowmap_scratch_bytes(int64_t T, int32_t K, int32_t E);
 gq4_status gq4_rowmap(const int32_t *idx, int64_t T, int32_t K, int32_t E, int32_t *cnt,
                       int32_t *offs, int32_t *row_tok, int32_t *row_slot, int32_t *slot_row,
