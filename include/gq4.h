@@ -30,7 +30,9 @@
  *     quantisation calls also take any gs that is a multiple of 8 with in % 8 == 0
  *     (partial last groups included) on generic kernels; moe_expert_ffn needs gs = 64.
  *     Other shapes return GQ4_ERR_UNSUPPORTED (the host packer accepts any shape).
- *   - No call keeps global mutable state, reads environment variables or throws.
+ *   - No call reads environment variables or throws.  No call keeps global mutable
+ *     state, with one exception: moe_expert_ffn_noalloc uses a library-owned device
+ *     array per GPU and caches that array's device address per device (see its entry).
  */
 #ifndef GQ4_H
 #define GQ4_H
@@ -42,7 +44,7 @@
 extern "C" {
 #endif
 
-#define GQ4_ABI_VERSION 5u
+#define GQ4_ABI_VERSION 6u
 
 typedef struct CUstream_st *gq4_stream_t; /* binary-compatible with cudaStream_t */
 typedef struct CUevent_st *gq4_event_t;   /* binary-compatible with cudaEvent_t */
@@ -90,6 +92,7 @@ typedef struct {
     int32_t *n_active; /* [1] number of experts with cnt > 0 */
     int32_t *active;   /* [E] those experts, ascending */
     int32_t *status;   /* [1] device status word (gq4_status bits, see moe_expert_ffn) */
+    uint16_t *h;       /* [T*K][F] bf16 gate+up output silu(g)*u, row r = row-map row r */
 } gq4_routing;
 
 /* ABI version of the loaded library (GQ4_ABI_VERSION at build time).  The Python
@@ -127,7 +130,12 @@ gq4_status gq4_upload(const uint8_t *packed_host, const float *scales_host, int6
                       void *d_w, size_t d_w_bytes, float *d_s, size_t d_s_bytes,
                       gq4_stream_t stream, gq4_tensor *desc);
 
-/* Fill *desc for device data already laid out as above (no copy). */
+/* Fill *desc for device data already laid out as above (no copy).  The descriptor
+ * carries gs and ng with the pointers so that every launch site indexes the O*ng scale
+ * array by group (colibri PR #298, "fmt=4 CUDA attention crash -- root cause": the fix
+ * threaded w->gs and w->ng, which the uploaded tensor already carried, through every
+ * launch; "Summary / Changes": tensor_upload allocates O*ng scales for fmt=4).  Expert
+ * strides are set to the tight sizes; a caller with padded experts edits them after. */
 gq4_status gq4_tensor_init(const void *d_w, const float *d_s, int64_t out, int64_t in,
                            int32_t gs, int32_t n_experts, gq4_tensor *desc);
 
@@ -177,6 +185,14 @@ gq4_status gq4_rowmap(const int32_t *idx, int64_t T, int32_t K, int32_t E, int32
  *   y[t] = sum_j wts[t][j] * Wd_e (silu(Wg_e x_t) * (Wu_e x_t)),  e = idx[t][j]
  * with the router, the on-device row map, the fused gate+up (h rounded to bf16), the
  * down projection and the weighted scatter-add all on the GPU, no host round trip.
+ * Sources: colibri PR #298, "Summary / Changes" (the fmt=4 expert matmuls and the fused
+ * grouped gate+up pair, matmul_i4_grouped_pair, which halved expert-matmul time) and
+ * "implementation complete but blocked" (top-K by K passes over taken flags, the grouped
+ * down projection); pxq_llama.cpp release notes 2026-09-02, "Device-side MoE row map"
+ * (the token -> expert table built on the device with histogram, scan and fill, because
+ * a host-built table forced a device-to-host sync per layer).  The top-K softmax
+ * renormalised over the chosen experts, SiLU(gate)*up and the weighted sum of the K
+ * expert outputs complete the layer as the method statement gives it.
  *   Wg, Wu: E stacked [F][H]; Wd: E stacked [H][F]; logits device f32 [T][E];
  *   x device bf16 [T][H]; y device f32 [T][H] (overwritten); ws device workspace of
  *   moe_expert_ffn_workspace_bytes(T, E, K, H, F) bytes; 1 <= K <= E <= 1024.
@@ -207,8 +223,10 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
                           int32_t E, int32_t K, float *y, void *ws, size_t ws_bytes,
                           gq4_event_t const *stage_events, gq4_stream_t stream);
 
-/* Device pointers of the routing tables inside a workspace used by moe_expert_ffn with
- * the same (T, E, K, H, F). */
+/* Device pointers of the routing tables and of h (the bf16 gate+up output, in row-map
+ * order) inside a workspace used by moe_expert_ffn with the same (T, E, K, H, F).  h is
+ * computed in a fixed order on every path, so repeated calls on the same inputs give
+ * the same h bit for bit (y is not: its K contributions meet through float atomics). */
 gq4_status moe_expert_ffn_routing(void *ws, size_t ws_bytes, int64_t T, int32_t E, int32_t K,
                                   int64_t H, int64_t F, gq4_routing *out);
 
@@ -298,6 +316,12 @@ gq4_status gq4_mla_absorb_v(const gq4_tensor *W, int32_t n_heads, int32_t d_nope
  * gq4_selftest_wait_timeout or of moe_expert_ffn_noalloc -- into *status_host (0, or the
  * OR of GQ4_ERR_NONFINITE_LOGIT, GQ4_ERR_TIMEOUT, ... the kernels raised).  Synchronous:
  * it returns after all work queued on `stream` before it has finished.
+ * Data-dependent errors stay on the device so that no compute call has to synchronise
+ * (pxq_llama.cpp release notes 2026-09-02, "Device-side MoE row map": a device-to-host
+ * sync inside the per-layer loop was the cost the on-device table removed); the caller
+ * reads the word with this call when it chooses.  An out-of-range index becomes a status
+ * bit rather than a fault (colibri PR #298, "fmt=4 CUDA attention crash -- root cause":
+ * a wrong scale index became a GPU memory fault and a system crash).
  *   status_dev: 16-byte aligned device int32; status_host: host int32.
  *   Returns GQ4_ERR_CUDA when the copy or the synchronisation fails (for example after an
  *   earlier launch failed on the stream). */

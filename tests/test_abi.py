@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = gq4.lib()
-    assert lib.gq4_abi_version() == 5
+    assert lib.gq4_abi_version() == 6
     for st in range(10):
         assert lib.gq4_status_string(st).decode()
     assert lib.gq4_status_string(77) == b"unknown status"

@@ -65,7 +65,10 @@ def test_matvec_and_gate_up_stay_in_bounds(O, I, T, gs):
     assert intact(buf, _words(h))
 
 
-@pytest.mark.parametrize("T,E,K,H,F", [(5, 4, 2, 256, 192), (40, 8, 4, 384, 192), (70, 3, 2, 128, 64)])
+@pytest.mark.parametrize("T,E,K,H,F", [(5, 4, 2, 256, 192), (40, 8, 4, 384, 192), (70, 3, 2, 128, 64),
+                                       # tensor-core kernels: 45 rows per expert (not a multiple
+                                       # of 16), and 60-80 rows beside decode-path experts
+                                       (45, 2, 2, 256, 256), (100, 5, 2, 512, 256)])
 def test_moe_output_stays_in_bounds(T, E, K, H, F):
     cfg = synth.MoEConfig(f"guard_t{T}_e{E}", T=T, H=H, E=E, F=F, K=K, seed=T + E)
     parts = {n: [getattr(cfg, n)(e) for e in range(E)] for n in ("gate", "up", "down")}
@@ -76,6 +79,8 @@ def test_moe_output_stays_in_bounds(T, E, K, H, F):
                                bf16_to_torch(cfg.x()), K, y=y)
     assert ws.status() == 0
     assert intact(buf, _words(y))
+    if H % 256 == 0 and F % 256 == 0 and T >= gq4.MOE_LARGE_MIN_ROWS:
+        assert int(ws.routing()["cnt"].max()) >= gq4.MOE_LARGE_MIN_ROWS  # reaches the tensor cores
 
 
 def test_row_ops_and_mla_stay_in_bounds():

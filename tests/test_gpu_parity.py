@@ -226,15 +226,26 @@ def _toy(T, E, K, H=128, F=128, seed=3, **kw):
     return synth.MoEConfig(f"toy_t{T}_e{E}_k{K}", T=T, H=H, E=E, F=F, K=K, seed=seed, **kw)
 
 
+def _takes_tensor_cores(cfg, cnt):
+    """True when moe_expert_ffn sends at least one expert of this call to the tensor-core
+    kernels: T >= GQ4_MOE_LARGE_MIN_ROWS, H a multiple of 128 with 4-group stages of the
+    gate/up rows (H % 256 == 0) and of the down rows (F % 256 == 0), and an expert with at
+    least GQ4_MOE_LARGE_MIN_ROWS rows."""
+    lim = gq4.MOE_LARGE_MIN_ROWS
+    return cfg.T >= lim and cfg.H % 256 == 0 and cfg.F % 256 == 0 and int(cnt.max()) >= lim
+
+
 @pytest.mark.parametrize("T,E,K,H,F", [(5, 4, 2, 128, 128), (1, 1, 1, 64, 64), (3, 8, 8, 192, 256),
                                        (17, 16, 4, 256, 128), (40, 32, 8, 128, 192),
                                        (300, 16, 4, 128, 64),
-                                       # tensor-core path (experts with >= 33 rows), mixed with
-                                       # the decode path, multi-pass experts (> 192 rows)
+                                       # many rows per expert on shapes the tensor-core kernels
+                                       # do not take (H or F not a multiple of 256): the decode
+                                       # kernels in several column passes
                                        (64, 4, 2, 256, 128), (40, 8, 4, 384, 192), (300, 2, 1, 128, 64),
-                                       (500, 2, 2, 128, 128), (48, 4, 2, 192, 128), (130, 6, 3, 512, 256),
-                                       # passes of many sizes in one CTA (activation byte ring laps)
+                                       (500, 2, 2, 128, 128), (48, 4, 2, 192, 128),
                                        (600, 12, 3, 256, 128), (1000, 8, 2, 128, 64),
+                                       # tensor-core path beside the decode path
+                                       (130, 6, 3, 512, 256),
                                        # TMA-fed decode kernel for gate+up and down (H, F multiples
                                        # of 256), alone and beside the tensor-core path
                                        (12, 16, 4, 256, 256), (30, 8, 8, 512, 256), (20, 64, 8, 256, 512),
@@ -245,6 +256,36 @@ def test_moe_small_full_oracle(T, E, K, H, F):
     s = MoESet(_toy(T, E, K, H, F))
     y, ws = s.run()
     assert ws.status() == 0
+    s.check(y, ws, np.arange(T))
+
+
+@pytest.mark.parametrize("T,E,K,H,F,n_hot,min_max_rows", [
+    # one hot expert takes nearly every token (> 512 rows: several tensor-core passes)
+    # and the others 200-400 rows each
+    (600, 4, 2, 256, 256, 1, 513),
+    # 200-300 rows per expert: one full pass and a ragged second one
+    (500, 4, 2, 256, 256, 0, 193),
+    # rows just above the decode/tensor-core split, not multiples of 16
+    (45, 2, 2, 256, 256, 0, 45),
+    # wider matrices, 1000+ rows on the hot expert, down tiles of several M tiles
+    (1100, 6, 2, 512, 768, 1, 513),
+    # experts just above the split (33..46 rows) beside decode-path experts (15..32)
+    (400, 24, 2, 256, 512, 0, 33)])
+def test_moe_tensor_core_cases(T, E, K, H, F, n_hot, min_max_rows):
+    """Workloads that reach the tensor-core kernels (asserted from the row map, so the
+    labels cannot go stale), with experts of many row counts: several passes, ragged
+    last passes, counts that are not multiples of 16.  Two calls must give the same h
+    bit for bit."""
+    cfg = synth.MoEConfig(f"tc_t{T}_e{E}_k{K}_h{H}_f{F}", T=T, H=H, E=E, F=F, K=K, seed=T + 7 * E,
+                          n_hot=n_hot, hot_bias=4.0 if n_hot else 0.0)
+    s = MoESet(cfg)
+    y, ws = s.run()
+    assert ws.status() == 0
+    cnt = ws.routing()["cnt"].cpu().numpy()
+    assert _takes_tensor_cores(cfg, cnt)
+    assert int(cnt.max()) >= min_max_rows
+    _, ws2 = s.run()
+    assert torch.equal(ws2.routing()["h"], ws.routing()["h"])
     s.check(y, ws, np.arange(T))
 
 
@@ -271,29 +312,38 @@ def test_moe_decode_full_size(moe_decode):
 
 def test_moe_batched_decode_full_size():
     """The benchmark's workload (32 tokens, 256 experts of 6144 x 2048, top-8, skewed
-    routing), in the benchmark's launch configuration; routing and the row map in
-    full, the output on a seeded sample of 8 tokens."""
+    routing), in the benchmark's launch configuration; routing, the row map and the
+    output of every token against the oracle.  A second call gives the same h bit for
+    bit (fixed summation order) and y within rounding (float atomics in the scatter-add)."""
     s = MoESet(synth.MOE_BATCHED)
     y, ws = s.run()
     assert ws.status() == 0
-    y2, _ = s.run()  # a second call reuses nothing stale
+    y2, ws2 = s.run()  # a second call reuses nothing stale
+    assert torch.equal(ws2.routing()["h"], ws.routing()["h"])
     assert np.allclose(y, y2, rtol=1e-5, atol=1e-3)
-    tokens = np.sort(np.random.default_rng(1003).choice(32, 8, replace=False))
-    s.check(y, ws, tokens)
+    del ws2
+    s.check(y, ws, np.arange(synth.MOE_BATCHED.T))
     del s
     torch.cuda.empty_cache()
 
 
 def test_moe_prefill_full_size():
-    """4096 tokens over all 256 experts; routing and the row map in full, the output
-    on 32 tokens of the seeded 256-token sample (a wrong h row of any expert shows up
-    in the tokens routed to it, so the sample is wide enough to catch a fault in a
-    fraction of the tensor-core tiles)."""
+    """4096 tokens over all 256 experts in the benchmark's launch configuration:
+    routing and the row map in full, the output on the whole seeded 256-token sample.
+    Three calls in a row (after the other MoE cases of this file) must give the same h
+    bit for bit -- every path computes h in a fixed order, so a race in the tensor-core
+    pipeline shows up as a difference -- and y within rounding."""
     s = MoESet(synth.MOE_PREFILL)
     y, ws = s.run()
     assert ws.status() == 0
-    tokens = synth.MOE_PREFILL.sample_tokens()[::8]
-    s.check(y, ws, tokens)
+    h0 = ws.routing()["h"]
+    for _ in range(2):
+        y2, ws2 = s.run()
+        assert ws2.status() == 0
+        assert torch.equal(ws2.routing()["h"], h0)
+        assert np.allclose(y2, y, rtol=1e-5, atol=1e-4)
+        del ws2
+    s.check(y, ws, synth.MOE_PREFILL.sample_tokens())
     del s
     torch.cuda.empty_cache()
 
@@ -304,7 +354,8 @@ def test_moe_prefill_512_tokens_32_experts():
     s = MoESet(synth.MOE_PREFILL_E32)
     y, ws = s.run()
     assert ws.status() == 0
-    y2, _ = s.run()
+    y2, ws2 = s.run()
+    assert torch.equal(ws2.routing()["h"], ws.routing()["h"])
     assert np.allclose(y, y2, rtol=1e-5, atol=1e-4)
     s.check(y, ws, synth.MOE_PREFILL_E32.sample_tokens())
     del s

@@ -348,6 +348,61 @@ def test_rowmap_vs_stable_argsort(T, E, K):
         assert np.all(flat[seg] == e) and np.all(np.diff(seg) > 0)
 
 
+# ---------------------------------------------------------------- row L1 norms (tolerance scale)
+# The per-element acceptance bound is 2e-3 * ||w_row||_1 * max|x| ("compare against the
+# sum of |terms|", the maintainer's oracle reply on colibri PR #298); these pins fix the
+# norm the bound is built from.
+def _dense_any(p, s, I, gs):
+    """Independent numpy decode for any group size and odd widths (low nibble first,
+    two's complement, scale of column k = s[:, k // gs])."""
+    b = p.astype(np.int16)
+    nib = np.empty((p.shape[0], 2 * p.shape[1]), np.int16)
+    nib[:, 0::2] = b & 15
+    nib[:, 1::2] = b >> 4
+    q = np.where(nib >= 8, nib - 16, nib)[:, :I].astype(np.float64)
+    cols = np.arange(I) // gs
+    return q * s.astype(np.float64)[:, cols]
+
+
+@pytest.mark.parametrize("O,I,gs", [(7, 64, 64), (5, 200, 64), (3, 129, 16), (4, 96, 128),
+                                    (6, 33, 64), (2, 512, 64), (9, 250, 48)])
+def test_row_l1_vs_numpy_dense(O, I, gs):
+    r = np.random.default_rng(O * 1000 + I)
+    q = r.integers(-8, 8, size=(O, I)).astype(np.int8)
+    ng = -(-I // gs)
+    # signed scales: the norm is over |s * q|, so a negative scale must count positively
+    s = (r.uniform(0.002, 0.02, size=(O, ng)) * r.choice([-1.0, 1.0], size=(O, ng))).astype(np.float32)
+    p = oracle.pack(q)
+    got = oracle.row_l1(p, s, I, gs)
+    want = np.abs(_dense_any(p, s, I, gs)).sum(1)
+    assert np.allclose(got, want, rtol=1e-12, atol=0)
+    # the matvec's own bound is the same norm times max|x| of each token
+    x = r.standard_normal((2, I)).astype(np.float32)
+    _, b = oracle.matvec(p, s, x, gs)
+    assert np.allclose(b, want[None, :] * np.abs(x).max(1)[:, None], rtol=1e-12, atol=0)
+
+
+def test_row_l1_exact_power_of_two_scales():
+    """Hand-worked norms with scales 2^-j, exact in fp64: a row of all -8 over 3 groups,
+    an alternating +7/-8 row, a row of zeros, and a row whose second group is the only
+    nonzero one (catches a norm summed over the wrong axis or without |.|)."""
+    I, gs = 192, 64
+    q = np.zeros((4, I), np.int8)
+    q[0] = -8
+    q[1, 0::2], q[1, 1::2] = 7, -8
+    q[3, 64:128] = 3
+    s = np.array([[2.0 ** -3, 2.0 ** -4, 2.0 ** -5],
+                  [-2.0 ** -2, 2.0 ** -2, -2.0 ** -2],
+                  [1.0, 1.0, 1.0],
+                  [2.0 ** -7, -2.0 ** -6, 2.0 ** -7]], np.float32)
+    got = oracle.row_l1(oracle.pack(q), s, I, gs)
+    want = [8 * 64 * (2.0 ** -3 + 2.0 ** -4 + 2.0 ** -5),
+            (7 + 8) * 32 * 3 * 2.0 ** -2,
+            0.0,
+            3 * 64 * 2.0 ** -6]
+    assert list(got) == want
+
+
 # ---------------------------------------------------------------- a6-a8: MoE
 def _dense(p, s, I, gs=64):
     b = p.astype(np.int16)

@@ -711,6 +711,7 @@ gq4_status moe_expert_ffn_routing(void *ws, size_t ws_bytes, int64_t T, int32_t 
     out->n_active = at<int32_t>(ws, L.n_active);
     out->active = at<int32_t>(ws, L.active);
     out->status = at<int32_t>(ws, L.status);
+    out->h = at<uint16_t>(ws, L.h);
     return GQ4_OK;
 }
 
@@ -935,16 +936,25 @@ extern "C" gq4_status moe_expert_ffn_noalloc(const gq4_tensor *Wg, const gq4_ten
     if (status_out && !aligned16(status_out)) return GQ4_ERR_ALIGN;
     const MoeLayout L = moe_layout(T, E, K, Wg->in, Wg->out);
     if (L.total > GQ4_NOALLOC_SCRATCH_BYTES) return GQ4_ERR_WORKSPACE;
-    void *ws = nullptr;
-    gq4_status st = noalloc_scratch(&ws);
-    if (st != GQ4_OK) return st;
     if (!logits || !x || !y) return GQ4_ERR_NULL;
+    gq4_status st = GQ4_OK;
     if (status_out) {
+        // the status word is written after the layer: it must not sit inside any input
+        // or output (weights and scales included), or the copy would overwrite them
+        if ((st = check_tensor(Wg, 1)) != GQ4_OK || (st = check_tensor(Wu, 1)) != GQ4_OK ||
+            (st = check_tensor(Wd, 1)) != GQ4_OK)
+            return st;
         const Range sr = rng(status_out, 4);
-        if (overlap(sr, rng(y, (size_t)T * Wg->in * 4)) || overlap(sr, rng(logits, (size_t)T * E * 4)) ||
-            overlap(sr, rng(x, (size_t)T * Wg->in * 2)))
-            return GQ4_ERR_ALIAS;
+        const Range others[] = {rng(y, (size_t)T * Wg->in * 4), rng(logits, (size_t)T * E * 4),
+                                rng(x, (size_t)T * Wg->in * 2),
+                                rng(Wg->w, tensor_w_bytes(Wg)), rng(Wg->s, tensor_s_bytes(Wg)),
+                                rng(Wu->w, tensor_w_bytes(Wu)), rng(Wu->s, tensor_s_bytes(Wu)),
+                                rng(Wd->w, tensor_w_bytes(Wd)), rng(Wd->s, tensor_s_bytes(Wd))};
+        for (const Range &r : others)
+            if (overlap(sr, r)) return GQ4_ERR_ALIAS;
     }
+    void *ws = nullptr;
+    if ((st = noalloc_scratch(&ws)) != GQ4_OK) return st;
     // moe_expert_ffn validates everything else and clears the status word itself
     st = moe_expert_ffn(Wg, Wu, Wd, logits, x, xdt, T, E, K, y, ws, GQ4_NOALLOC_SCRATCH_BYTES, nullptr,
                         stream);

@@ -16,7 +16,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgq4.so")
-ABI_VERSION = 5
+ABI_VERSION = 6
 MOE_STAGE_EVENTS = 6
 MOE_LARGE_MIN_ROWS = 33  # GQ4_MOE_LARGE_MIN_ROWS
 NOALLOC_SCRATCH_BYTES = 16 << 20  # GQ4_NOALLOC_SCRATCH_BYTES
@@ -42,7 +42,7 @@ class TensorDesc(ctypes.Structure):
 class RoutingDesc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("idx", "wts", "cnt", "offs", "row_tok", "row_slot", "slot_row", "n_active",
-                 "active", "status")]
+                 "active", "status", "h")]
 
 
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
@@ -272,7 +272,8 @@ class MoEWorkspace:
         self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
 
     def routing(self) -> dict:
-        """Views of the routing tables (device int32/f32 tensors) after a call."""
+        """Views of the routing tables (device int32/f32 tensors) and of h (bf16 bit
+        patterns as int16, [T*K][F], row-map order) after a call."""
         T, E, K, H, F = self.shape
         r = RoutingDesc()
         _check(_lib.moe_expert_ffn_routing(self.buf.data_ptr(), self.nbytes, T, E, K, H, F,
@@ -289,7 +290,8 @@ class MoEWorkspace:
                     cnt=view(r.cnt, E, torch.int32), offs=view(r.offs, E + 1, torch.int32),
                     row_tok=view(r.row_tok, n, torch.int32), row_slot=view(r.row_slot, n, torch.int32),
                     slot_row=view(r.slot_row, n, torch.int32), n_active=view(r.n_active, 1, torch.int32),
-                    active=view(r.active, E, torch.int32), status=view(r.status, 1, torch.int32))
+                    active=view(r.active, E, torch.int32), status=view(r.status, 1, torch.int32),
+                    h=self.buf[r.h - base:r.h - base + n * F * 2].view(torch.int16).view(n, F))
 
     def status(self, stream=None) -> int:
         T, E, K, H, F = self.shape
