@@ -9,6 +9,17 @@ top-8, skewed routing (16 hot experts get +3 on logits of variance 2).
 
 Prints one JSON line (rank 0).  N > 1 (under torchrun): independent replicas, one per
 GPU (the layer has no exchange step), weak scaling, time = max over ranks.
+
+The line's headline is the chosen workload (default: batched decode).  At N = 1 it also
+carries a "configs" object with every other workload of the specification, each timed
+the same way (CUDA-graph replay between L2 flushes, device events; an end-to-end figure
+through the public API with host buffers; the roofline of its dominant kernel):
+  * MoE decode, 1 token, hidden 4096, 128 experts of 1536, top-8;
+  * MoE prefill, 4096 tokens, hidden 6144, 256 experts of 2048, top-8;
+  * the dense gq4_matvec sweep at batch 1 (4096x4096, 14336x4096, 4096x14336,
+    151936x4096);
+  * the single expert: gate+up+SiLU [2048][1024] and down [1024][2048] with f32 x.
+(--configs none skips them.)
 """
 from __future__ import annotations
 
@@ -48,6 +59,12 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+# Nominal B200 figures the metric is also quoted against: HBM3e 8 TB/s, dense bf16
+# tensor throughput 2.25 PFLOP/s.
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -55,6 +72,20 @@ def peaks():
             d = json.load(f)
         return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
     return 6650.0, 1590.0, "fallback"
+
+
+def roofline(bound, achieved, hbm, bf16, peak_kind):
+    """Roofline entry of one kernel: the fraction of the measured peak (copy bandwidth or
+    cuBLAS bf16) and of the nominal one (8 TB/s or 2.25 PFLOP/s)."""
+    if bound == "tensor":
+        r = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+             "peak_nominal": NOMINAL_BF16_TFLOPS}
+    else:
+        r = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "peak_nominal": NOMINAL_HBM_GBS}
+    r["frac"] = achieved / r["peak"]
+    r["frac_nominal"] = achieved / r["peak_nominal"]
+    r["peak_kind"] = peak_kind
+    return r
 
 
 class ClockSampler:
@@ -276,31 +307,11 @@ def run_reference(args, cfg, rank):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=synth.MOE_BATCHED.name, choices=list(synth.MOE_CONFIGS))
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
-    cfg = synth.MOE_CONFIGS[args.workload]
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        run_reference(args, cfg, rank)
-        return
-
+def moe_run(cfg, args, dev, world, local, with_cpu):
+    """Time one MoE workload: device-timed graph replays, the per-stage split, the
+    end-to-end figure through the public API, and the dominant kernel's roofline.
+    Returns the fields of its JSON entry."""
     import torch
-    import torch.distributed as dist
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     from weight_only_int4_gq4_b200 import gq4
 
     # ---- inputs resident in HBM (weights of all E experts, logits, x)
@@ -319,7 +330,6 @@ def main():
     ws = gq4.MoEWorkspace(cfg.T, cfg.E, cfg.K, cfg.H, cfg.F, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    n_slots = cfg.T * cfg.K
     NEV = gq4.MOE_STAGE_EVENTS
 
     def step(ev=None):
@@ -352,6 +362,7 @@ def main():
         graph.replay()
         graph_st.replay()
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     step_ms = np.zeros(args.steps)
@@ -407,12 +418,10 @@ def main():
     dom = max(busy or STAGES[1:], key=lambda k: t_stage[k])
     dbytes, dflops = work[dom]
     if dflops > 0:
-        roof = {"bound": "tensor", "achieved": dflops / (t_stage[dom] * 1e-3) / 1e12, "peak": bf16,
-                "unit": "TFLOP/s", "alg_flops_per_launch": dflops}
+        roof = roofline("tensor", dflops / (t_stage[dom] * 1e-3) / 1e12, hbm, bf16, peak_kind)
+        roof["alg_flops_per_launch"] = dflops
     else:
-        roof = {"bound": "hbm", "achieved": dbytes / (t_stage[dom] * 1e-3) / 1e9, "peak": hbm,
-                "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+        roof = roofline("hbm", dbytes / (t_stage[dom] * 1e-3) / 1e9, hbm, bf16, peak_kind)
     roof["alg_bytes_per_launch"] = dbytes
     traffic = None
     if os.path.exists(PROFILE_TRAFFIC):
@@ -422,36 +431,215 @@ def main():
         if rec and rec.get("source_hash") == kernel_source_hash():
             traffic = rec["bytes_per_launch"]
     roof["traffic"] = traffic
-    roof = {"kernel": kern[dom], "stage": dom, "peak_kind": peak_kind, **roof}
+    roof = {"kernel": kern[dom], "stage": dom, **roof}
     step_bytes = sum(b for b, _ in work.values())
+    step_flops = sum(f for _, f in work.values())
     per_expert = 2 * per_matrix_bytes(cfg.F, cfg.H) + per_matrix_bytes(cfg.H, cfg.F)
     n_active = split["n_small"] + split["n_large"]
+    out = {
+        "value": job_tokens_per_s(world, cfg.T, ms), "unit": "tokens/s", "ms_per_step": ms,
+        "ms_p10_p50_p90": [float(v) for v in np.percentile(step_ms, [10, 50, 90])],
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "F": cfg.F, "K": cfg.K,
+                   "gs": 64, "distinct_experts": n_active, "experts_tensor_core": split["n_large"],
+                   "parallelism": f"replicas x{world}",
+                   "launch": "value: CUDA-graph replay of one moe_expert_ffn call, events around the "
+                             "replay; stage_ms: a second graph with the call's stage events; "
+                             "e2e: direct calls",
+                   "l2": f"{L2_FLUSH_BYTES >> 20} MiB flush between steps; touched weights "
+                         f"{n_active * per_expert / 1e9:.2f} GB/step"},
+        "hbm_gbs_step": step_bytes / (ms * 1e-3) / 1e9,
+        "stage_ms": t_stage,
+        "roofline": roof,
+        "e2e": {"value": job_tokens_per_s(world, cfg.T, e2e), "unit": "tokens/s",
+                "h2d_bytes_per_step": x_h.nbytes + lg_h.nbytes, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
+        "gpu_launches": launches_per_step(cfg, split) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if step_flops > 0:
+        out["tflops_step"] = step_flops / (ms * 1e-3) / 1e12
+    if with_cpu:
+        out["cpu_baseline"] = cpu_baseline(cfg)
+    del Wg, Wu, Wd, ws, flush
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_replays(fn, steps, warmup, flush):
+    """Milliseconds per replay of one captured call (mean, p10/p50/p90), L2 flushed
+    between replays, events on the launching stream around each replay."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(warmup):
+        g.replay()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    del g
+    return float(np.mean(ts)), [float(v) for v in np.percentile(ts, [10, 50, 90])]
+
+
+def time_e2e(fn, steps, warmup, flush):
+    """Milliseconds per direct call including the caller's host<->device copies (fn does
+    the copies and the call), events around each step."""
+    import torch
+    stream = torch.cuda.current_stream()
+    ts = []
+    for i in range(warmup + steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        if i >= warmup:
+            ts.append(a.elapsed_time(b))
+    return float(np.mean(ts))
+
+
+def dense_run(args, dev):
+    """The dense gq4_matvec sweep (batch 1, bf16 x): per shape the device time of the
+    call, its HBM roofline (packed nibbles + scales + x read, y written) and the end-to-end
+    time with x copied in from pinned host memory and y copied out."""
+    import torch
+    from weight_only_int4_gq4_b200 import gq4
+    hbm, bf16, kind = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    res = {}
+    for O, I in synth.DENSE_SHAPES:
+        p, sc, xb = synth.dense_matvec(O, I)
+        W = gq4.upload(p, sc)
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.empty(1, O, dtype=torch.float32, device=dev)
+        ms, pct = time_replays(lambda: gq4.matvec(W, x, y), args.steps, args.warmup, flush)
+        x_pin = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        y_pin = torch.empty(1, O, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_pin, non_blocking=True)
+            gq4.matvec(W, x, y)
+            y_pin.copy_(y, non_blocking=True)
+        e2e = time_e2e(e2e_step, args.steps, args.warmup, flush)
+        nbytes = per_matrix_bytes(O, I) + I * 2 + O * 4
+        res[f"{O}x{I}"] = {
+            "value": 1.0 / (ms * 1e-3), "unit": "tokens/s", "us": ms * 1e3, "us_p10_p50_p90": [v * 1e3 for v in pct],
+            "roofline": {"kernel": "gq4_matvec", **roofline("hbm", nbytes / (ms * 1e-3) / 1e9, hbm, bf16, kind),
+                         "alg_bytes_per_launch": nbytes, "traffic": None},
+            "e2e": {"value": 1.0 / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": I * 2,
+                    "d2h_bytes_per_step": O * 4}}
+        del W
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def single_expert_run(args, dev):
+    """The single-expert layer: gate+up+SiLU ([2048][1024] each) then down ([1024][2048])
+    on one f32 token, device time of the pair of calls and end to end."""
+    import torch
+    from weight_only_int4_gq4_b200 import gq4
+    se = synth.SingleExpert()
+    hbm, bf16, kind = peaks()
+    Wg = gq4.upload(gq4.pack(se.qg), se.sg)
+    Wu = gq4.upload(gq4.pack(se.qu), se.su)
+    Wd = gq4.upload(gq4.pack(se.qd), se.sd)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    x = torch.from_numpy(se.x).to(dev)
+    h = torch.empty(1, se.F, dtype=torch.float32, device=dev)
+    y = torch.empty(1, se.H, dtype=torch.float32, device=dev)
+
+    def layer():
+        gq4.gate_up_silu(Wg, Wu, x, h)
+        gq4.matvec(Wd, h, y)
+    ms, pct = time_replays(layer, args.steps, args.warmup, flush)
+    x_pin = torch.from_numpy(se.x).pin_memory()
+    y_pin = torch.empty(1, se.H, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        x.copy_(x_pin, non_blocking=True)
+        layer()
+        y_pin.copy_(y, non_blocking=True)
+    e2e = time_e2e(e2e_step, args.steps, args.warmup, flush)
+    nbytes = 2 * per_matrix_bytes(se.F, se.H) + per_matrix_bytes(se.H, se.F) + 4 * (2 * se.H + 2 * se.F)
+    out = {"value": 1.0 / (ms * 1e-3), "unit": "tokens/s", "us": ms * 1e3, "us_p10_p50_p90": [v * 1e3 for v in pct],
+           "roofline": {"kernel": "gq4_gate_up_silu + gq4_matvec (2 launches)",
+                        **roofline("hbm", nbytes / (ms * 1e-3) / 1e9, hbm, bf16, kind),
+                        "alg_bytes_per_launch": nbytes, "traffic": None,
+                        "note": "3.5 MB of weights: latency-bound, far below any bandwidth roof"},
+           "e2e": {"value": 1.0 / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": se.H * 4,
+                   "d2h_bytes_per_step": se.H * 4}}
+    del Wg, Wu, Wd, flush
+    torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=synth.MOE_BATCHED.name, choices=list(synth.MOE_CONFIGS))
+    ap.add_argument("--configs", default="all", choices=["all", "none"],
+                    help="also time the other workloads of the specification (N = 1 only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = synth.MOE_CONFIGS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    head = moe_run(cfg, args, dev, world, local, with_cpu=not args.no_cpu_baseline and world == 1)
+    configs = None
+    if args.configs == "all" and world == 1:
+        configs = {}
+        for c in (synth.MOE_DECODE, synth.MOE_BATCHED, synth.MOE_PREFILL):
+            if c.name != cfg.name:
+                configs[c.name] = moe_run(c, args, dev, world, local, with_cpu=False)
+        configs["dense_matvec_t1_bf16"] = dense_run(args, dev)
+        configs["single_expert_f32_1024_2048"] = single_expert_run(args, dev)
 
     if rank == 0:
         line = {
-            "metric": "expert-FFN tokens/s (MoE layer, 1 B200)", "value": job_tokens_per_s(world, cfg.T, ms),
+            "metric": "expert-FFN tokens/s (MoE layer, 1 B200)", "value": head["value"],
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms, "ms_p10_p50_p90": [float(v) for v in np.percentile(step_ms, [10, 50, 90])],
+            "ms_per_step": head["ms_per_step"], "ms_p10_p50_p90": head["ms_p10_p50_p90"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "F": cfg.F, "K": cfg.K,
-                       "gs": 64, "distinct_experts": n_active, "experts_tensor_core": split["n_large"],
-                       "parallelism": f"replicas x{world}",
-                       "launch": "value: CUDA-graph replay of one moe_expert_ffn call, events around the "
-                                 "replay; stage_ms: a second graph with the call's stage events; "
-                                 "e2e: direct calls",
-                       "l2": f"{L2_FLUSH_BYTES >> 20} MiB flush between steps; touched weights "
-                             f"{n_active * per_expert / 1e9:.2f} GB/step"},
-            "hbm_gbs_step": step_bytes / (ms * 1e-3) / 1e9,
-            "stage_ms": t_stage,
-            "roofline": roof,
-            "e2e": {"value": job_tokens_per_s(world, cfg.T, e2e), "unit": "tokens/s",
-                    "h2d_bytes_per_step": x_h.nbytes + lg_h.nbytes, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
-            "gpu_launches": launches_per_step(cfg, split) * args.steps,
-            "clocks": clk.summary(),
+            "config": head["config"],
+            "hbm_gbs_step": head["hbm_gbs_step"],
+            "stage_ms": head["stage_ms"],
+            "roofline": head["roofline"],
+            "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"],
+            "clocks": head["clocks"],
         }
-        if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(cfg)
+        if "cpu_baseline" in head:
+            line["cpu_baseline"] = head["cpu_baseline"]
+        if configs is not None:
+            line["configs"] = configs
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
