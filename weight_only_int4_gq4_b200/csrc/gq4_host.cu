@@ -434,6 +434,10 @@ gq4_status launch_tc(const CUtensorMap &w0, const CUtensorMap &w1, const CUtenso
     auto kern = gq4_tc_kernel<MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes) != cudaSuccess)
         return GQ4_ERR_CUDA;
+    // the kernel's register split (setmaxnreg) must fit in what the launch allocates
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GQ4_ERR_CUDA;
+    if ((int64_t)fa.numRegs * kTcThreads < kTcRegsNeeded) return GQ4_ERR_UNSUPPORTED;
     const int grid = std::max(1, std::min(units_upper, sm_count()));
     kern<<<grid, kTcThreads, kTcSmemBytes, st>>>(w0, w1, x[0], x[1], x[2], x[3], p);
     return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;

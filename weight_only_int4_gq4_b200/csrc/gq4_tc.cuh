@@ -17,7 +17,7 @@
 // Warp roles (512 threads = 4 warpgroups, one CTA per SM, persistent over units):
 //   WG0  warp 0  TMA producer of the packed nibble tiles: 128 rows x 128 B (four groups,
 //                swizzle 128B) per stage in two 64-row boxes, 5-stage ring
-//        warp 1  TMEM allocation and the MMA issuer (one thread)
+//        warp 1  TMEM allocation and the MMA issuer (one elected lane of the warp)
 //        warp 2  TMA producer of the activation tiles (N <= 192 rows x 64 bf16, swizzle
 //                128B) as 128/64/32/16-row boxes, 4-stage ring; warp 3 idle
 //   (TMA cost is per request more than per byte: few large boxes keep the rings fed)
@@ -57,6 +57,10 @@ constexpr int kTcOffBar = kTcOffW + kTcWStages * kTcWBytes;
 constexpr int kTcSmemBytes = kTcOffBar + 512 + 1024;            // + 1024 for alignment
 static_assert(kTcSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kTcTmemCols = 512;                                // two N<=192 partials (power of 2)
+constexpr int kTcRegsLow = 48, kTcRegsHigh = 200;               // setmaxnreg split
+// registers the split needs from the launch: a launch with fewer per thread would leave
+// setmaxnreg.inc waiting forever, so the host refuses it (cudaFuncAttributes::numRegs)
+constexpr int kTcRegsNeeded = 256 * kTcRegsLow + 256 * kTcRegsHigh;
 constexpr int kStatusTimeout = 8;                               // GQ4_ERR_TIMEOUT
 
 struct TcParams {
@@ -170,16 +174,21 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 __device__ __forceinline__ uint32_t idesc_bf16_m128(int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                       uint32_t accumulate) {
+// D (+)= A * B (both from shared memory, descriptors), issued by one lane elected from
+// the converged calling warp.  ACC (accumulate into D) is a compile-time predicate.
+template <bool ACC>
+__device__ __forceinline__ void tc_mma_elect(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc) {
     asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate) : "memory");
+        "{\n .reg .pred e, p;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "n"(ACC ? 1 : 0) : "memory");
 }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(bar) : "memory");
+// tcgen05.commit (arrive on `bar` once this thread's MMAs are done) by the elected lane.
+__device__ __forceinline__ void tc_commit_elect(uint32_t bar) {
+    asm volatile(
+        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+        " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n"
+        ::"r"(bar) : "memory");
 }
 // tcgen05.ld writes its destination registers asynchronously, until tcgen05.wait::ld.
 // The compiler treats them as written by the load itself, so between a separate load and
@@ -272,7 +281,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
     const int n_units = (*p.n_large) * p.m_tiles;
 
     if (warp < 8) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 48;" ::: "memory");
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kTcRegsLow) : "memory");
       if (warp == 0 || warp == 2) {
         // ------------------------------------------------------------ TMA producers
         // warp 0: packed weights into the W ring; warp 2: activations into the X ring
@@ -327,7 +336,11 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
         __syncwarp();
       } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the loop (converged); lane 0 polls the barriers and one
+        // elected lane issues each MMA and commit.  The accumulate flag of each MMA is a
+        // compile-time predicate: computing it at run time just before the instruction
+        // made every issue cost ~210 cycles on B200 (measured), a third of the pipe's rate.
+        {
             uint32_t it = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
@@ -339,25 +352,28 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                     const uint32_t idesc = idesc_bf16_m128(N);
                     for (int G = 0; G < p.ng; ++G, ++it) {
                         const int xs = it % kTcXStages, as = it % kTcAStages, b = it & 1;
-                        ok = mbar_wait(xfull_bar(xs), (it / kTcXStages) & 1, abort_flag, p.status) &&
-                             mbar_wait(afull_bar(as), (it / kTcAStages) & 1, abort_flag, p.status) &&
-                             mbar_wait(pempty_bar(b), ((it >> 1) & 1) ^ 1, abort_flag, p.status);
+                        if (lane == 0)
+                            ok = mbar_wait(xfull_bar(xs), (it / kTcXStages) & 1, abort_flag, p.status) &&
+                                 mbar_wait(afull_bar(as), (it / kTcAStages) & 1, abort_flag, p.status) &&
+                                 mbar_wait(pempty_bar(b), ((it >> 1) & 1) ^ 1, abort_flag, p.status);
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t a_addr = sb + kTcOffA + as * kTcABytes;
                         const uint32_t x_addr = sb + kTcOffX + xs * kTcXBytes;
-                        #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma(tmem + b * 256, sw128_desc(a_addr + kk * 32),
-                                   sw128_desc(x_addr + kk * 32), idesc, kk > 0 ? 1u : 0u);
-                        tc_commit(pfull_bar(b));
-                        tc_commit(aempty_bar(as));
-                        tc_commit(xempty_bar(xs));
+                        const uint64_t ad = sw128_desc(a_addr), xd = sw128_desc(x_addr);
+                        tc_mma_elect<false>(tmem + b * 256, ad, xd, idesc);
+                        tc_mma_elect<true>(tmem + b * 256, ad + 2, xd + 2, idesc);
+                        tc_mma_elect<true>(tmem + b * 256, ad + 4, xd + 4, idesc);
+                        tc_mma_elect<true>(tmem + b * 256, ad + 6, xd + 6, idesc);
+                        tc_commit_elect(pfull_bar(b));
+                        tc_commit_elect(aempty_bar(as));
+                        tc_commit_elect(xempty_bar(xs));
                     }
                 }
             }
             // the last commits must have arrived before the CTA's shared memory is released
-            if (ok && it > 0) {
+            if (lane == 0 && ok && it > 0) {
                 const uint32_t j = it - 1;
                 mbar_wait(xempty_bar(j % kTcXStages), (j / kTcXStages) & 1, abort_flag, p.status);
                 mbar_wait(aempty_bar(j % kTcAStages), (j / kTcAStages) & 1, abort_flag, p.status);
@@ -421,7 +437,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
       }
     } else {
         // ------------------------------------------------------------ promotion warps
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kTcRegsHigh) : "memory");
         const int q = warp & 3;              // TMEM lane quarter this warp may access
         const int half = (warp - 8) >> 2;    // column half: 32-column chunks 2c + half
         const int lrow = 32 * q + lane;      // TMEM lane = A row
@@ -500,19 +516,25 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                 if (!ok) break;
                 // ---------------------------------------------------- epilogue
                 if (MODE == 0) {
-                    // even lane: gate row, odd lane: the up row of the same output f
+                    // even lane: gate row, odd lane: the up row of the same output f.  Per
+                    // pair of columns (j, j+1) the even lane finishes column j and the odd
+                    // lane column j+1: each sends its partner the value the partner lacks
                     const int f = mt * 64 + (lrow >> 1);
+                    const bool odd = lane & 1;
                     #pragma unroll
                     for (int c = 0; c < kTcChunks; ++c) {
                         const int col = 32 * (2 * c + half);
                         if (col < N) {
                             #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const float uv = __shfl_xor_sync(0xffffffffu, acc[c][j], 1);
-                                if (!(lane & 1) && col + j < nrows) {
-                                    const float g = acc[c][j];
+                            for (int j = 0; j < 32; j += 2) {
+                                const float send = odd ? acc[c][j] : acc[c][j + 1];
+                                const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                                const float g = odd ? recv : acc[c][j];
+                                const float uv = odd ? acc[c][j + 1] : recv;
+                                const int jj = col + j + (odd ? 1 : 0);
+                                if (jj < nrows) {
                                     const float hv = g / (1.0f + expf(-g)) * uv;
-                                    p.h[(int64_t)(row0 + n0 + col + j) * p.O + f] = (uint16_t)bf16_bits_rn(hv);
+                                    p.h[(int64_t)(row0 + n0 + jj) * p.O + f] = (uint16_t)bf16_bits_rn(hv);
                                 }
                             }
                         }
