@@ -31,8 +31,9 @@
  *     (partial last groups included) on generic kernels; moe_expert_ffn needs gs = 64.
  *     Other shapes return GQ4_ERR_UNSUPPORTED (the host packer accepts any shape).
  *   - No call reads environment variables or throws.  No call keeps global mutable
- *     state, with one exception: moe_expert_ffn_noalloc uses a library-owned device
- *     array per GPU and caches that array's device address per device (see its entry).
+ *     state, with two exceptions: moe_expert_ffn_noalloc uses a library-owned device
+ *     array per GPU and caches that array's device address per device (see its entry),
+ *     and the checked build keeps one bounds status word (gq4_bounds_status).
  */
 #ifndef GQ4_H
 #define GQ4_H
@@ -44,7 +45,7 @@
 extern "C" {
 #endif
 
-#define GQ4_ABI_VERSION 6u
+#define GQ4_ABI_VERSION 7u
 
 typedef struct CUstream_st *gq4_stream_t; /* binary-compatible with cudaStream_t */
 typedef struct CUevent_st *gq4_event_t;   /* binary-compatible with cudaEvent_t */
@@ -59,7 +60,8 @@ typedef enum {
     GQ4_ERR_WORKSPACE = 6,   /* workspace too small */
     GQ4_ERR_CUDA = 7,        /* a CUDA runtime call failed */
     GQ4_ERR_TIMEOUT = 8,     /* a bounded device wait gave up (see gq4_selftest_wait_timeout) */
-    GQ4_ERR_NONFINITE_LOGIT = 9 /* a router row held NaN/+inf, or no finite maximum */
+    GQ4_ERR_NONFINITE_LOGIT = 9, /* a router row held NaN/+inf, or no finite maximum */
+    GQ4_ERR_BOUNDS = 16      /* an index fell outside its array (checked build only) */
 } gq4_status;
 
 typedef enum { GQ4_F32 = 0, GQ4_BF16 = 1 } gq4_dtype;
@@ -364,6 +366,29 @@ gq4_status moe_expert_ffn_noalloc(const gq4_tensor *Wg, const gq4_tensor *Wu,
                                   const gq4_tensor *Wd, const float *logits, const void *x,
                                   gq4_dtype xdt, int64_t T, int32_t E, int32_t K, float *y,
                                   int32_t *status_out, gq4_stream_t stream);
+
+/* ---- checked build
+ * The bug class the source pages report is an index outside its array: the MLA absorb
+ * kernels read the O*ng scale array of a grouped tensor with a bare row index (colibri
+ * PR #298, "fmt=4 CUDA attention crash -- root cause"), and a shard's scale pointer was
+ * offset by rows instead of rows*ng (the maintainer's oracle reply).  A library built with
+ * GQ4_CHECKED defined (libgq4_checked.so) tests every weight, scale and activation-row
+ * index its kernels compute against the extent of its array -- taken from the tensor
+ * descriptors and the call's sizes -- before the access.  An index outside is not used:
+ * the access reads zeros (a copy that must deliver its bytes reads row 0 instead), the
+ * results are then not valid, and GQ4_ERR_BOUNDS is OR-ed into one library-wide bounds
+ * status word.  Nothing traps.  Outputs written through a valid index are unchanged.
+ * gq4_build_checked: 1 for a checked library, 0 otherwise.
+ * gq4_bounds_status: waits for `stream`, reads the bounds status word into *status_host
+ *   (0 or GQ4_ERR_BOUNDS; always 0 in an unchecked library) and clears it when `clear` is
+ *   non-zero.  The word is shared by every call on every stream of the process.
+ * gq4_selftest_bounds: launches, on `stream`, a test of `index` against `extent` that
+ *   accesses no memory, so that the reporting path can be tested without an out-of-range
+ *   access; in a checked library index outside [0, extent) raises GQ4_ERR_BOUNDS.
+ *   GQ4_ERR_SHAPE for a negative extent. */
+int32_t gq4_build_checked(void);
+gq4_status gq4_bounds_status(int32_t clear, gq4_stream_t stream, int32_t *status_host);
+gq4_status gq4_selftest_bounds(int64_t index, int64_t extent, gq4_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = gq4.lib()
-    assert lib.gq4_abi_version() == 6
+    assert lib.gq4_abi_version() == 7
     for st in range(10):
         assert lib.gq4_status_string(st).decode()
     assert lib.gq4_status_string(77) == b"unknown status"
@@ -225,3 +225,21 @@ def test_sync_status_argument_checks():
     assert L.gq4_sync_status(0x100000, None, None) == gq4.ERR_NULL
     assert L.gq4_sync_status(0x100004, None, ctypes.byref(v)) == gq4.ERR_ALIGN
     assert v.value == -1
+
+
+def test_checked_library_loads_and_exports_every_symbol():
+    """The bounds-checked build exports the same ABI and says it is checked (host calls
+    only; no GPU needed)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib = os.path.join(root, "weight_only_int4_gq4_b200", "libgq4_checked.so")
+    assert os.path.exists(lib), "build it with `python -m weight_only_int4_gq4_b200.build --checked`"
+    code = ("from weight_only_int4_gq4_b200 import gq4\n"
+            "assert gq4.build_checked() == 1\n"
+            "assert all(hasattr(gq4.lib(), n) for n in gq4.EXPORTED)\n"
+            "print('ok')\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=dict(os.environ, GQ4_LIBRARY=lib),
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr

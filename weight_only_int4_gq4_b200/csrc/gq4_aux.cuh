@@ -109,8 +109,9 @@ __global__ void __launch_bounds__(256) gq4_dequant_rows_kernel(const uint32_t *d
             }
             continue;
         }
-        const uint32_t v = __ldg(dw + row * wpr + wi);
-        const float s = __ldg(ds + row * ng + (wi * 8) / gs);
+        const int64_t wix = row * wpr + wi, six = row * ng + (wi * 8) / gs;
+        const uint32_t v = in_bounds(wix, n_weight_rows * wpr) ? __ldg(dw + wix) : 0u;
+        const float s = in_bounds(six, n_weight_rows * (int64_t)ng) ? __ldg(ds + six) : 0.f;
         const float a = alpha ? alpha[j] : 1.f;
         float r[8];
         #pragma unroll
@@ -189,8 +190,10 @@ __global__ void __launch_bounds__(256) gq4_generic_kernel(const uint32_t *dw0, c
                 #pragma unroll
                 for (int t = 0; t < kGenMaxTok; ++t) { p0[t] = 0.f; p1[t] = 0.f; }
                 for (int wi = 0; wi < words; ++wi) {
-                    const uint32_t v0 = __ldg(dw0 + row * wpr + w0 + wi);
-                    const uint32_t v1 = MODE == 1 ? __ldg(dw1 + row * wpr + w0 + wi) : 0u;
+                    const int64_t wix = row * wpr + w0 + wi;
+                    const bool wok = in_bounds(wix, n_weight_rows * wpr);
+                    const uint32_t v0 = wok ? __ldg(dw0 + wix) : 0u;
+                    const uint32_t v1 = MODE == 1 && wok ? __ldg(dw1 + wix) : 0u;
                     const int64_t k = (w0 + wi) * 8;
                     #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -206,8 +209,10 @@ __global__ void __launch_bounds__(256) gq4_generic_kernel(const uint32_t *dw0, c
                         }
                     }
                 }
-                const float s0 = __ldg(ds0 + row * ng + g);
-                const float s1 = MODE == 1 ? __ldg(ds1 + row * ng + g) : 0.f;
+                const int64_t six = row * ng + g;
+                const bool sok = in_bounds(six, n_weight_rows * (int64_t)ng);
+                const float s0 = sok ? __ldg(ds0 + six) : 0.f;
+                const float s1 = MODE == 1 && sok ? __ldg(ds1 + six) : 0.f;
                 #pragma unroll
                 for (int t = 0; t < kGenMaxTok; ++t) {
                     acc0[t] = fmaf(s0, p0[t], acc0[t]);

@@ -66,4 +66,38 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return g / (1.0f + expf(-g)) * u;
 }
 
+// ---- checked build (GQ4_CHECKED) ------------------------------------------------------
+// The bug class the pages report is an index outside its array: a scale read with a row
+// index on an O*ng scale array (colibri PR #298, "fmt=4 CUDA attention crash -- root
+// cause") and a shard's scale pointer offset by rows instead of rows*ng (the
+// maintainer's oracle reply).  Built with GQ4_CHECKED, the kernels test every weight,
+// scale and activation-row index they compute against the extent of its array before
+// the access.  An index outside is not used -- the access reads zeros, or a copy that
+// must still deliver its bytes reads row 0 instead -- and GQ4_ERR_BOUNDS is OR-ed into the
+// library's bounds status word (gq4_bounds_status reads it).  Nothing traps.  Without the
+// flag the tests compile away.
+#ifdef GQ4_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+constexpr int32_t kStatusBounds = 16;  // GQ4_ERR_BOUNDS
+__device__ int32_t g_bounds_status;    // OR of kStatusBounds raised since the last clear
+
+// True when 0 <= i < n (always true without GQ4_CHECKED).
+__device__ __forceinline__ bool in_bounds(int64_t i, int64_t n) {
+    if constexpr (!kChecked) {
+        return true;
+    } else {
+        if (i >= 0 && i < n) return true;
+        atomicOr(&g_bounds_status, kStatusBounds);
+        return false;
+    }
+}
+
+// Self-test of the mechanism: tests index i against extent n and accesses nothing.
+__global__ void gq4_bounds_selftest_kernel(int64_t i, int64_t n) {
+    if (threadIdx.x == 0) (void)in_bounds(i, n);
+}
+
 }  // namespace gq4

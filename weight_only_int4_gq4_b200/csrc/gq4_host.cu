@@ -67,6 +67,20 @@ inline size_t tensor_s_bytes(const gq4_tensor *t) {
     return ((size_t)(t->n_experts - 1) * t->expert_stride_s + (size_t)t->out * t->ng) * 4;
 }
 
+// Array extents the checked build tests indexes against: the weight and scale arrays of
+// t0 (and t1, the smaller of the two), the rows of the activation array, the experts.
+void set_extents(SkinnyParams &p, const gq4_tensor *t0, const gq4_tensor *t1, int64_t x_rows, int n_exp) {
+    size_t wb = tensor_w_bytes(t0), sb = tensor_s_bytes(t0);
+    if (t1) {
+        wb = std::min(wb, tensor_w_bytes(t1));
+        sb = std::min(sb, tensor_s_bytes(t1));
+    }
+    p.w_bytes = (int64_t)wb;
+    p.s_count = (int64_t)(sb / 4);
+    p.x_rows = x_rows;
+    p.n_exp = n_exp;
+}
+
 int sm_count() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
@@ -494,6 +508,7 @@ const char *gq4_status_string(int status) {
         case GQ4_ERR_CUDA: return "CUDA runtime error";
         case GQ4_ERR_TIMEOUT: return "a bounded device wait gave up";
         case GQ4_ERR_NONFINITE_LOGIT: return "router logits hold NaN/+inf or no finite maximum";
+        case GQ4_ERR_BOUNDS: return "an index fell outside its array (checked build)";
         default: return "unknown status";
     }
 }
@@ -592,6 +607,7 @@ gq4_status gq4_matvec(const gq4_tensor *W, const void *x, gq4_dtype xdt, int64_t
     p.row_tiles = (int)((W->out + 15) / 16);
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.y = y;
+    set_extents(p, W, nullptr, n_tok, 1);
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
     if (check_tensor(W, 1) != GQ4_OK) {  // another group size or a partial last group
         const int sh = wide_group_shift(W);
@@ -631,6 +647,7 @@ gq4_status gq4_gate_up_silu(const gq4_tensor *Wg, const gq4_tensor *Wu, const vo
     p.row_tiles = (int)((Wg->out + 15) / 16);
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.h = h;
+    set_extents(p, Wg, Wu, n_tok, 1);
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
     if (check_tensor(Wg, 1) != GQ4_OK || check_tensor(Wu, 1) != GQ4_OK) {  // general group size
         const int sh = wide_group_shift(Wg);
@@ -823,6 +840,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     pg.x = x; pg.xdt = 1; pg.n_tok = (int)T;
     pg.h = at<void>(ws, L.h);
     pg.zero_ptr = y; pg.zero_n = T * H;
+    set_extents(pg, Wg, Wu, T, E);
     if ((T * H) % 4) return GQ4_ERR_SHAPE;
     const int small_cols = (int)std::min<int64_t>(max_cols, tc ? kLargeMin - 1 : max_cols);
     const bool band = small_cols >= kBandMinCols;
@@ -845,7 +863,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
         gq4_gather_rows_kernel<<<sm_count() * 4, 256, 0, s>>>((const uint4 *)x, at<int32_t>(ws, L.row_tok),
                                                              at<int32_t>(ws, L.offs), at<int32_t>(ws, L.cnt),
                                                              lists.n_large, lists.large, chunks,
-                                                             at<uint4>(ws, L.xg));
+                                                             at<uint4>(ws, L.xg), T, E);
         if (cudaGetLastError() != cudaSuccess) return GQ4_ERR_CUDA;
         const uint64_t rows_gu = (uint64_t)(Wg->n_experts - 1) * (Wg->expert_stride_w / (H / 2)) + F;
         const uint64_t rows_d = (uint64_t)(Wd->n_experts - 1) * (Wd->expert_stride_w / (F / 2)) + H;
@@ -865,10 +883,13 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
         tp.status = at<int32_t>(ws, L.status);
         tp.h = at<uint16_t>(ws, L.h);
         tp.y = y;
+        tp.n_exp = E;
+        tp.n_tok = (int)T;
         TcParams tg = tp;
         tg.s0 = Wg->s; tg.s1 = Wu->s; tg.estride_s = Wg->expert_stride_s;
         tg.O = (int)F; tg.I = (int)H; tg.ng = Wg->ng; tg.m_tiles = (int)(F / 64);
         tg.estride_rows = (int)(Wg->expert_stride_w / (H / 2));
+        tg.s_count = (int64_t)(std::min(tensor_s_bytes(Wg), tensor_s_bytes(Wu)) / 4);
         st = launch_tc<0>(tm_g, tm_u, tm_x, tg, max_large * tg.m_tiles, s);
         if (st != GQ4_OK) return st;
     }
@@ -881,6 +902,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     pd.row_tiles = (int)((H + 15) / 16);
     pd.x = at<void>(ws, L.h); pd.xdt = 1; pd.n_tok = (int)T;
     pd.y = y;
+    set_extents(pd, Wd, nullptr, T * K, E);
     if (stream_usable(Wd))
         st = launch_stream<kMoeDown>(stream_mats(Wd, nullptr), pd, small_cols, max_active, status, s);
     else
@@ -894,6 +916,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
         td.s0 = Wd->s; td.s1 = Wd->s; td.estride_s = Wd->expert_stride_s;
         td.O = (int)H; td.I = (int)F; td.ng = Wd->ng; td.m_tiles = (int)(H / 128);
         td.estride_rows = (int)(Wd->expert_stride_w / (F / 2));
+        td.s_count = (int64_t)(tensor_s_bytes(Wd) / 4);
         st = launch_tc<1>(tm_d, tm_d, tm_h, td, max_large * td.m_tiles, s);
     }
     mark(5);
@@ -1067,6 +1090,7 @@ extern "C" gq4_status gq4_matvec_rows(const gq4_tensor *W, const int32_t *idx, i
     p.row_tiles = (int)((n_sel + 15) / 16);
     p.x = x; p.xdt = (int)xdt; p.n_tok = (int)n_tok;
     p.y = y;
+    set_extents(p, W, nullptr, n_tok, 1);
     const int cols = (int)(xdt == GQ4_F32 ? 3 * n_tok : n_tok);
     return launch_skinny<kMatvec>(p, cols, xdt == GQ4_F32, p.row_tiles, S(stream));
 }
@@ -1168,4 +1192,31 @@ extern "C" gq4_status gq4_sync_status(const int32_t *status_dev, gq4_stream_t st
     if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return GQ4_ERR_CUDA;
     *status_host = v;
     return GQ4_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Checked build: bounds status word and its self-test
+// ---------------------------------------------------------------------------------------
+extern "C" int32_t gq4_build_checked(void) { return kChecked ? 1 : 0; }
+
+extern "C" gq4_status gq4_bounds_status(int32_t clear, gq4_stream_t stream, int32_t *status_host) {
+    if (!status_host) return GQ4_ERR_NULL;
+    int32_t v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_bounds_status, 4, 0, cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess)
+        return GQ4_ERR_CUDA;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return GQ4_ERR_CUDA;
+    if (clear) {
+        const int32_t zero = 0;
+        if (cudaMemcpyToSymbolAsync(g_bounds_status, &zero, 4, 0, cudaMemcpyHostToDevice, S(stream)) != cudaSuccess ||
+            cudaStreamSynchronize(S(stream)) != cudaSuccess)
+            return GQ4_ERR_CUDA;
+    }
+    *status_host = v;
+    return GQ4_OK;
+}
+
+extern "C" gq4_status gq4_selftest_bounds(int64_t index, int64_t extent, gq4_stream_t stream) {
+    if (extent < 0) return GQ4_ERR_SHAPE;
+    gq4_bounds_selftest_kernel<<<1, 32, 0, S(stream)>>>(index, extent);
+    return cudaGetLastError() == cudaSuccess ? GQ4_OK : GQ4_ERR_CUDA;
 }

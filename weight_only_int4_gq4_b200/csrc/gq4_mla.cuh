@@ -75,8 +75,9 @@ __global__ void __launch_bounds__(kMlaThreads) gq4_mla_q_kernel(const uint32_t *
         #pragma unroll 4
         for (int d = d0 + split; d < d1; d += nsplit) {
             const int64_t row = (int64_t)h * D + d;
-            const uint32_t v = __ldg(w + row * W + j);
-            const float sc = __ldg(s + row * ng + g);
+            const int64_t wix = row * W + j, six = row * ng + g;
+            const uint32_t v = in_bounds(wix, (int64_t)nh * D * W) ? __ldg(w + wix) : 0u;
+            const float sc = in_bounds(six, (int64_t)nh * D * ng) ? __ldg(s + six) : 0.f;
             float qv[8];
             #pragma unroll
             for (int m = 0; m < 8; ++m) qv[m] = (float)dev_q(v, dev_slot(m));
@@ -158,8 +159,9 @@ __global__ void __launch_bounds__(kMlaThreads) gq4_mla_v_kernel(const uint32_t *
         #pragma unroll
         for (int r = 0; r < kMlaVRowsPerWarp; ++r) {
             const int64_t row = (int64_t)h * D + dn + v0 + min(r, nv - 1);
-            word[r] = __ldg(w + row * W + j);
-            sc[r] = __ldg(s + row * ng + (8 * j) / gs);
+            const int64_t wix = row * W + j, six = row * ng + (8 * j) / gs;
+            word[r] = in_bounds(wix, (int64_t)nh * D * W) ? __ldg(w + wix) : 0u;
+            sc[r] = in_bounds(six, (int64_t)nh * D * ng) ? __ldg(s + six) : 0.f;
         }
         float qv[kMlaVRowsPerWarp][8];  // the words decoded once, used by every token
         #pragma unroll

@@ -303,17 +303,19 @@ namespace gq4 {
 // kernels read only those rows).  One warp per (large expert, row) pair.
 __global__ void gq4_gather_rows_kernel(const uint4 *x, const int32_t *row_tok, const int32_t *offs,
                                        const int32_t *cnt, const int32_t *n_large, const int32_t *large,
-                                       int chunks_per_row, uint4 *xg) {
+                                       int chunks_per_row, uint4 *xg, int64_t x_rows, int n_exp) {
     const int nl = *n_large;
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
     int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     for (int a = 0; a < nl; ++a) {
         const int e = large[a];
+        if (!in_bounds(e, n_exp)) continue;  // the same for every warp
         const int r0 = offs[e], n = cnt[e];
         for (; w < n; w += warps) {
             const int r = r0 + w;
-            const uint4 *src = x + (int64_t)row_tok[r] * chunks_per_row;
+            const int64_t xr = row_tok[r];
+            const uint4 *src = x + (in_bounds(xr, x_rows) ? xr : 0) * chunks_per_row;
             uint4 *dst = xg + (int64_t)r * chunks_per_row;
             for (int c = lane; c < chunks_per_row; c += 32) dst[c] = src[c];
         }

@@ -63,6 +63,10 @@ struct SkinnyParams {
     int sng;
     const int32_t *rows;
     int n_out;
+    // extents for the checked build (GQ4_CHECKED): bytes of the weight array (all experts),
+    // floats of the scale array, rows of the activation array, experts of the call
+    int64_t w_bytes, s_count, x_rows;
+    int n_exp;
 };
 
 template <int MODE>
@@ -88,12 +92,12 @@ __device__ __forceinline__ void skinny_stage(const SkinnyParams &p, char *xs, in
         uint32_t w[8];
         if (MODE == kMoeGateUp || MODE == kMoeDown || p.xdt == 1) {
             const uint16_t *src;
-            if (MODE == kMoeGateUp)
-                src = (const uint16_t *)p.x + (int64_t)p.row_tok[row0 + c] * p.I;
-            else if (MODE == kMoeDown)
-                src = (const uint16_t *)p.x + (int64_t)(row0 + c) * p.I;
-            else
-                src = (const uint16_t *)p.x + (int64_t)c * p.I;
+            int64_t xr;
+            if (MODE == kMoeGateUp) xr = p.row_tok[row0 + c];
+            else if (MODE == kMoeDown) xr = row0 + c;
+            else xr = c;
+            if (!in_bounds(xr, p.x_rows)) xr = 0;
+            src = (const uint16_t *)p.x + xr * p.I;
             const uint4 a = *((const uint4 *)(src + piece * 16));
             const uint4 b = *((const uint4 *)(src + piece * 16 + 8));
             w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
@@ -163,6 +167,7 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
             const int a = u / p.row_tiles;
             rt = u - a * p.row_tiles;
             e = p.active[a];
+            if (!in_bounds(e, p.n_exp)) continue;  // uniform across the block
             row0 = p.offs[e];
             cols = p.cnt[e];
         } else {
@@ -214,10 +219,16 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
                             const uint8_t *Wm = m ? W1 : W0;
                             const float *Sm = m ? S1 : S0;
                             const int64_t off = (int64_t)G * 32 + t * 8;
-                            wa[m][q] = (ok && vA) ? ldg_stream_u2(Wm + (int64_t)rA * rb + off) : make_uint2(0, 0);
-                            wb[m][q] = (ok && vB) ? ldg_stream_u2(Wm + (int64_t)rB * rb + off) : make_uint2(0, 0);
-                            sa[m][q] = (ok && vA) ? ldg_f32(Sm + (int64_t)rA * sng + (G >> p.gshift)) : 0.f;
-                            sb[m][q] = (ok && vB) ? ldg_f32(Sm + (int64_t)rB * sng + (G >> p.gshift)) : 0.f;
+                            // byte and float offsets from the tensor's start (checked build)
+                            const int64_t wbase = (int64_t)e * p.estride_w, sbase = (int64_t)e * p.estride_s;
+                            const bool wA = ok && vA && in_bounds(wbase + (int64_t)rA * rb + off + 7, p.w_bytes);
+                            const bool wB = ok && vB && in_bounds(wbase + (int64_t)rB * rb + off + 7, p.w_bytes);
+                            const bool cA = ok && vA && in_bounds(sbase + (int64_t)rA * sng + (G >> p.gshift), p.s_count);
+                            const bool cB = ok && vB && in_bounds(sbase + (int64_t)rB * sng + (G >> p.gshift), p.s_count);
+                            wa[m][q] = wA ? ldg_stream_u2(Wm + (int64_t)rA * rb + off) : make_uint2(0, 0);
+                            wb[m][q] = wB ? ldg_stream_u2(Wm + (int64_t)rB * rb + off) : make_uint2(0, 0);
+                            sa[m][q] = cA ? ldg_f32(Sm + (int64_t)rA * sng + (G >> p.gshift)) : 0.f;
+                            sb[m][q] = cB ? ldg_f32(Sm + (int64_t)rB * sng + (G >> p.gshift)) : 0.f;
                         }
                     }
                     #pragma unroll
@@ -322,7 +333,8 @@ __global__ void __launch_bounds__(256) gq4_skinny_kernel(const SkinnyParams p) {
                         } else {  // kMoeDown: weighted scatter-add into y
                             const int r = row0 + c;
                             const float wt = p.wts[p.row_slot[r]];
-                            atomicAdd(p.y + (int64_t)p.row_tok[r] * p.O + o, wt * v[0]);
+                            const int tok = p.row_tok[r];
+                            if (in_bounds(tok, p.n_tok)) atomicAdd(p.y + (int64_t)tok * p.O + o, wt * v[0]);
                         }
                     }
                 }
@@ -429,6 +441,7 @@ __global__ void __launch_bounds__(256) gq4_band_kernel(const SkinnyParams p, int
             const int a = u / bands;
             band = u - a * bands;
             e = p.active[a];
+            if (!in_bounds(e, p.n_exp)) continue;  // uniform across the block
             row0 = p.offs[e];
             cols = p.cnt[e];
         }
@@ -450,14 +463,15 @@ __global__ void __launch_bounds__(256) gq4_band_kernel(const SkinnyParams p, int
                         const uint8_t *Wm = m ? W1 : W0;
                         const float *Sm = m ? S1 : S0;
                         const int row = rt * 16 + (lane >> 1);
-                        const bool rv = row < p.O;
-                        const uint8_t *src = Wm + (int64_t)(rv ? row : 0) * rb + (int64_t)G * 32 + (lane & 1) * 16;
+                        const int64_t woff = (int64_t)row * rb + (int64_t)G * 32 + (lane & 1) * 16;
+                        const bool rv = row < p.O && in_bounds((int64_t)e * p.estride_w + woff + 15, p.w_bytes);
+                        const uint8_t *src = Wm + (rv ? woff : 0);
                         cp_async16(smem_addr(st + m * 576 + (lane >> 1) * 32 + (lane & 1) * 16), src, rv ? 16u : 0u);
                         if (lane < 16) {
                             const int srow = rt * 16 + lane;
-                            const bool sv = srow < p.O;
-                            cp_async4(smem_addr(st + m * 576 + 512 + lane * 4), Sm + (int64_t)(sv ? srow : 0) * p.ng + G,
-                                      sv ? 4u : 0u);
+                            const int64_t soff = (int64_t)srow * p.ng + G;
+                            const bool sv = srow < p.O && in_bounds((int64_t)e * p.estride_s + soff, p.s_count);
+                            cp_async4(smem_addr(st + m * 576 + 512 + lane * 4), Sm + (sv ? soff : 0), sv ? 4u : 0u);
                         }
                     }
                 }
@@ -473,13 +487,12 @@ __global__ void __launch_bounds__(256) gq4_band_kernel(const SkinnyParams p, int
                     __syncwarp();
                     for (int r = lane; r < nc; r += 32) {
                         const int col = c0 + r;
-                        const uint16_t *src;
-                        if (MODE == kMoeGateUp)
-                            src = (const uint16_t *)p.x + (int64_t)p.row_tok[row0 + col] * p.I + k0;
-                        else if (MODE == kMoeDown)
-                            src = (const uint16_t *)p.x + (int64_t)(row0 + col) * p.I + k0;
-                        else
-                            src = (const uint16_t *)p.x + (int64_t)col * p.I + k0;
+                        int64_t xr;
+                        if (MODE == kMoeGateUp) xr = p.row_tok[row0 + col];
+                        else if (MODE == kMoeDown) xr = row0 + col;
+                        else xr = col;
+                        if (!in_bounds(xr, p.x_rows)) xr = 0;  // the copy must still deliver its bytes
+                        const uint16_t *src = (const uint16_t *)p.x + xr * p.I + k0;
                         bulk_g2s(smem_addr(xbuf + ((c & 1) * kBandMaxCols + r) * xstride), src, kn * 2, bar);
                     }
                 }
@@ -583,7 +596,9 @@ __global__ void __launch_bounds__(256) gq4_band_kernel(const SkinnyParams p, int
                                 (uint16_t)bf16_bits_rn(silu_mul(acc[0][n][i], acc[PAIR - 1][n][i]));
                         } else {
                             const int r = row0 + c;
-                            atomicAdd(p.y + (int64_t)p.row_tok[r] * p.O + o, p.wts[p.row_slot[r]] * acc[0][n][i]);
+                            const int tok = p.row_tok[r];
+                            if (in_bounds(tok, p.n_tok))
+                                atomicAdd(p.y + (int64_t)tok * p.O + o, p.wts[p.row_slot[r]] * acc[0][n][i]);
                         }
                     }
                 }

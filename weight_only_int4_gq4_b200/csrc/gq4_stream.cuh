@@ -210,6 +210,7 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
                 const int ai = u / bands;
                 band = u - ai * bands;
                 e = p.active[ai];
+                if (!in_bounds(e, p.n_exp)) e = 0;  // the stages must still be delivered
                 row0 = p.offs[e];
                 cols = p.cnt[e];
             }
@@ -218,12 +219,12 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
                 const int nc = min(PW, cols - c0);
                 const uint16_t *xrow = nullptr;  // this lane's activation row
                 if (lane < nc) {
-                    if (MODE == kMoeGateUp)
-                        xrow = (const uint16_t *)p.x + (int64_t)p.row_tok[row0 + c0 + lane] * p.I;
-                    else if (MODE == kMoeDown)
-                        xrow = (const uint16_t *)p.x + (int64_t)(row0 + c0 + lane) * p.I;
-                    else
-                        xrow = (const uint16_t *)p.x + (int64_t)(c0 + lane) * p.I;
+                    int64_t xr;
+                    if (MODE == kMoeGateUp) xr = p.row_tok[row0 + c0 + lane];
+                    else if (MODE == kMoeDown) xr = row0 + c0 + lane;
+                    else xr = c0 + lane;
+                    if (!in_bounds(xr, p.x_rows)) xr = 0;  // the copy must still deliver its bytes
+                    xrow = (const uint16_t *)p.x + xr * p.I;
                 }
                 const uint32_t tx = (uint32_t)(XOFF + nc * 512);
                 for (int k = 0; k < nst; ++k) {
@@ -271,6 +272,7 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
                 const int ai = u / bands;
                 band = u - ai * bands;
                 e = p.active[ai];
+                if (kChecked && (e < 0 || e >= p.n_exp)) e = 0;  // as the producer substituted
                 row0 = p.offs[e];
                 cols = p.cnt[e];
             }
@@ -358,7 +360,9 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
                                     (uint16_t)bf16_bits_rn(silu_mul(v0[n][i], v1[n][i]));
                             } else {
                                 const int r = row0 + c;
-                                atomicAdd(p.y + (int64_t)p.row_tok[r] * p.O + o, p.wts[p.row_slot[r]] * v0[n][i]);
+                                const int tok = p.row_tok[r];
+                                if (in_bounds(tok, p.n_tok))
+                                    atomicAdd(p.y + (int64_t)tok * p.O + o, p.wts[p.row_slot[r]] * v0[n][i]);
                             }
                         }
                     }

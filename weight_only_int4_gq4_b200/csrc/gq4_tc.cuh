@@ -75,6 +75,10 @@ struct TcParams {
     uint16_t *h;         // gate+up output, bf16 [T*K][O] in row-map order
     float *y;            // down output [T][O], accumulated
     int32_t *status;     // device status word
+    // extents for the checked build (GQ4_CHECKED): floats of the scale arrays, experts
+    // of the call, tokens (rows of y)
+    int64_t s_count;
+    int n_exp, n_tok;
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -224,6 +228,13 @@ __device__ __forceinline__ uint64_t splat2(float s) {
     return r;
 }
 
+// Expert of large-list entry a; in the checked build an entry outside [0, n_exp) raises
+// GQ4_ERR_BOUNDS and stands for expert 0, the same in every role of the CTA.
+__device__ __forceinline__ int tc_expert(const int32_t *large, int n_exp, int a) {
+    const int e = large[a];
+    return in_bounds(e, n_exp) ? e : 0;
+}
+
 // ---------------------------------------------------------------- the kernel
 template <int MODE>  // 0: gate+up with SiLU(g)*u -> h (bf16); 1: down -> y += w * D
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -292,7 +303,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
             bool ok = true;
             for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
                 const int a = u / p.m_tiles, mt = u - a * p.m_tiles;
-                const int e = p.large[a];
+                const int e = tc_expert(p.large, p.n_exp, a);
                 const int row0 = p.offs[e], cnt = p.cnt[e];
                 const int wrow = e * p.estride_rows + (MODE == 0 ? mt * 64 : mt * 128);
                 for (int n0 = 0; ok && n0 < cnt; n0 += kTcMaxN) {
@@ -345,7 +356,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
             bool ok = true;
             for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
                 const int a = u / p.m_tiles;
-                const int e = p.large[a];
+                const int e = tc_expert(p.large, p.n_exp, a);
                 const int cnt = p.cnt[e];
                 for (int n0 = 0; ok && n0 < cnt; n0 += kTcMaxN) {
                     const int N = (min(kTcMaxN, cnt - n0) + 15) & ~15;
@@ -393,7 +404,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
         uint32_t it = 0, wit = 0;  // group counter, weight-stage counter
         bool ok = true;
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-            const int e = p.large[u / p.m_tiles];
+            const int e = tc_expert(p.large, p.n_exp, u / p.m_tiles);
             const int cnt = p.cnt[e];
             for (int n0 = 0; ok && n0 < cnt; n0 += kTcMaxN) {
                 for (int G = 0; G < p.ng; ++G, ++it) {
@@ -447,14 +458,17 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
 
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
             const int a = u / p.m_tiles, mt = u - a * p.m_tiles;
-            const int e = p.large[a];
+            const int e = tc_expert(p.large, p.n_exp, a);
             const int row0 = p.offs[e], cnt = p.cnt[e];
-            const float *srow;  // the scale row of this thread's TMEM lane
-            if (MODE == 0)
-                srow = ((lrow & 1) ? p.s1 : p.s0) + (int64_t)e * p.estride_s +
-                       (int64_t)(mt * 64 + (lrow >> 1)) * p.ng;
-            else
-                srow = p.s0 + (int64_t)e * p.estride_s + (int64_t)(mt * 128 + lrow) * p.ng;
+            // the scale row of this thread's TMEM lane (offset in floats from the array start)
+            const int64_t soff = (int64_t)e * p.estride_s +
+                                 (int64_t)(MODE == 0 ? mt * 64 + (lrow >> 1) : mt * 128 + lrow) * p.ng;
+            const float *srow = ((MODE == 0 && (lrow & 1)) ? p.s1 : p.s0) + soff;
+            const int64_t s_count = p.s_count;
+            auto scales4 = [srow, soff, s_count](int k) {  // scales of groups k..k+3
+                return in_bounds(soff + k + 3, s_count) ? *(const float4 *)(srow + k)
+                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            };
             for (int n0 = 0; ok && n0 < cnt; n0 += kTcMaxN) {
                 const int nrows = min(kTcMaxN, cnt - n0);
                 const int N = (nrows + 15) & ~15;
@@ -463,14 +477,14 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                     #pragma unroll
                     for (int j = 0; j < 32; ++j) acc[c][j] = 0.f;
                 // scales four groups at a time, prefetched one float4 ahead (ng % 4 == 0)
-                float4 s_cur = *(const float4 *)srow;
-                float4 s_next = p.ng > 4 ? *(const float4 *)(srow + 4) : s_cur;
+                float4 s_cur = scales4(0);
+                float4 s_next = p.ng > 4 ? scales4(4) : s_cur;
                 for (int G = 0; G < p.ng; ++G, ++it) {
                     const int gq = G & 3;
                     const float sc = gq == 0 ? s_cur.x : gq == 1 ? s_cur.y : gq == 2 ? s_cur.z : s_cur.w;
                     if (gq == 3) {
                         s_cur = s_next;
-                        if (G + 5 < p.ng) s_next = *(const float4 *)(srow + G + 5);
+                        if (G + 5 < p.ng) s_next = scales4(G + 5);
                     }
                     const int b = it & 1;
                     if (!(ok = mbar_wait(pfull_bar(b), (it >> 1) & 1, abort_flag, p.status))) break;
@@ -552,12 +566,13 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                                 const int rr = row0 + n0 + col + lane;
                                 tok_l = p.row_tok[rr];
                                 wt_l = p.wts[p.row_slot[rr]];
+                                if (!in_bounds(tok_l, p.n_tok)) tok_l = -1;
                             }
                             #pragma unroll
                             for (int j = 0; j < 32; ++j) {
                                 const int tok = __shfl_sync(0xffffffffu, tok_l, j);
                                 const float wt = __shfl_sync(0xffffffffu, wt_l, j);
-                                if (col + j < nrows) atomicAdd(p.y + (int64_t)tok * p.O + o, wt * acc[c][j]);
+                                if (col + j < nrows && tok >= 0) atomicAdd(p.y + (int64_t)tok * p.O + o, wt * acc[c][j]);
                             }
                         }
                     }

@@ -3,7 +3,8 @@
 Argument marshalling only: every step of the computation runs in the CUDA kernels of
 the library.  PyTorch provides device memory and the current CUDA stream.  Importing
 this module loads the library and raises if it is missing or of another ABI version;
-there is no fallback.
+there is no fallback.  GQ4_LIBRARY, when set, names another build of the same library to
+load instead (the bounds-checked build, libgq4_checked.so).
 """
 from __future__ import annotations
 
@@ -15,19 +16,21 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libgq4.so")
-ABI_VERSION = 6
+LIB_PATH = os.environ.get("GQ4_LIBRARY") or os.path.join(_HERE, "libgq4.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "libgq4_checked.so")
+ABI_VERSION = 7
 MOE_STAGE_EVENTS = 6
 MOE_LARGE_MIN_ROWS = 33  # GQ4_MOE_LARGE_MIN_ROWS
 NOALLOC_SCRATCH_BYTES = 16 << 20  # GQ4_NOALLOC_SCRATCH_BYTES
 
 OK, ERR_NULL, ERR_ALIGN, ERR_SHAPE, ERR_UNSUPPORTED, ERR_ALIAS, ERR_WORKSPACE, ERR_CUDA, \
     ERR_TIMEOUT, ERR_NONFINITE_LOGIT = range(10)
+ERR_BOUNDS = 16
 F32, BF16 = 0, 1
 
 if not os.path.exists(LIB_PATH):
     raise RuntimeError(
-        f"libgq4.so not found at {LIB_PATH}: build it with "
+        f"{os.path.basename(LIB_PATH)} not found at {LIB_PATH}: build it with "
         "`python -m weight_only_int4_gq4_b200.build` (nvcc, sm_100a)")
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -76,6 +79,9 @@ _SIGS = {
     "gq4_mla_absorb_v": ([_TP, _I32, _I32, _I32, _P, ctypes.c_int, _I64, _P, _P], ctypes.c_int),
     "gq4_selftest_wait_timeout": ([ctypes.c_uint32, _P, _P], ctypes.c_int),
     "gq4_sync_status": ([_P, _P, ctypes.POINTER(_I32)], ctypes.c_int),
+    "gq4_build_checked": ([], ctypes.c_int32),
+    "gq4_bounds_status": ([_I32, _P, ctypes.POINTER(_I32)], ctypes.c_int),
+    "gq4_selftest_bounds": ([_I64, _I64, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -435,3 +441,21 @@ def sync_status(status: torch.Tensor, stream=None) -> int:
     v = _I32()
     _check(_lib.gq4_sync_status(status.data_ptr(), _stream(stream), ctypes.byref(v)), "gq4_sync_status")
     return v.value
+
+
+# ------------------------------------------------------------------ checked build
+def build_checked() -> bool:
+    """True when the loaded library is the bounds-checked build."""
+    return bool(_lib.gq4_build_checked())
+
+
+def bounds_status(clear: bool = True, stream=None) -> int:
+    """Waits for the stream and returns the bounds status word (0 or ERR_BOUNDS)."""
+    v = _I32()
+    _check(_lib.gq4_bounds_status(int(clear), _stream(stream), ctypes.byref(v)), "gq4_bounds_status")
+    return v.value
+
+
+def selftest_bounds(index: int, extent: int, stream=None) -> None:
+    """Tests index against extent on the device without any memory access."""
+    _check(_lib.gq4_selftest_bounds(index, extent, _stream(stream)), "gq4_selftest_bounds")
