@@ -8,17 +8,17 @@
 //   * q is turned into bf16 exactly (integers -8..7) by the math warps and written to
 //     shared memory in the 128-byte-swizzled K-major layout the MMA reads;
 //   * for each 64-wide group the MMA warp issues four M=128 x N x K=16 tcgen05.mma into
-//     one of two TMEM partial buffers (accumulate off for the first), then commits;
+//     one of three TMEM partial buffers (accumulate off for the first), then commits;
 //   * the math warps load the partial (tcgen05.ld), multiply it by the row's scale of
 //     that group and add it to running sums kept in registers ("promotion"), then free
-//     the buffer -- the MMA of group g+1 overlaps the promotion of group g.
+//     the buffer -- the MMAs of groups g+1 and g+2 overlap the promotion of group g.
 // TMEM lane = weight row, so the scale is one register per thread and group.
 //
 // Warp roles (512 threads = 4 warpgroups, one CTA per SM, persistent over units):
 //   WG0  warp 0  TMA producer of the packed nibble tiles: 128 rows x 128 B (four groups,
 //                swizzle 128B) per stage in two 64-row boxes, 5-stage ring
 //        warp 1  TMEM allocation and the MMA issuer (one elected lane of the warp)
-//        warp 2  TMA producer of the activation tiles (N <= 192 rows x 64 bf16, swizzle
+//        warp 2  TMA producer of the activation tiles (N <= 160 rows x 64 bf16, swizzle
 //                128B) as 128/64/32/16-row boxes, 4-stage ring; warp 3 idle
 //   (TMA cost is per request more than per byte: few large boxes keep the rings fed)
 //   WG1  warps 4-7   dequant: rows [32d, 32d+32) of the bf16 A tile, 3-slot ring
@@ -43,8 +43,9 @@ constexpr int kTcThreads = 512;
 constexpr int kTcWStages = 5;                                   // packed-weight ring, 4 groups/stage
 constexpr int kTcXStages = 4;                                   // activation ring, 1 group/stage
 constexpr int kTcAStages = 3;                                   // dequantised bf16 A tiles
-constexpr int kTcMaxN = 192;                                   // rows per pass (TMEM, registers)
-constexpr int kTcChunks = kTcMaxN / 64;                         // 32-column chunks per column half
+constexpr int kTcMaxN = 160;                                   // rows per pass (TMEM, registers)
+constexpr int kTcPBufs = 3;                                     // TMEM partial buffers of kTcMaxN columns
+constexpr int kTcChunks = (kTcMaxN + 63) / 64;                  // 32-column chunks per column half
 static_assert(kTcChunks == 3, "the promotion reads chunks 2c + half, c < 3");
 constexpr int kTcWGroups = 4;                                   // groups per weight stage
 constexpr int kTcWBytes = 128 * 32 * kTcWGroups;                // 128 rows x 256 nibbles
@@ -56,7 +57,8 @@ constexpr int kTcOffW = kTcOffA + kTcAStages * kTcABytes;
 constexpr int kTcOffBar = kTcOffW + kTcWStages * kTcWBytes;
 constexpr int kTcSmemBytes = kTcOffBar + 512 + 1024;            // + 1024 for alignment
 static_assert(kTcSmemBytes <= 232448, "shared memory per CTA");
-constexpr int kTcTmemCols = 512;                                // two N<=192 partials (power of 2)
+constexpr int kTcTmemCols = 512;                                // power of 2 >= kTcPBufs * kTcMaxN
+static_assert(kTcPBufs * kTcMaxN <= kTcTmemCols, "TMEM partial buffers");
 constexpr int kTcRegsLow = 48, kTcRegsHigh = 200;               // setmaxnreg split
 // registers the split needs from the launch: a launch with fewer per thread would leave
 // setmaxnreg.inc waiting forever, so the host refuses it (cudaFuncAttributes::numRegs)
@@ -254,9 +256,9 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
     auto afull_bar = [&](int a) { return bar0 + 272 + 8 * a; };
     auto aempty_bar = [&](int a) { return bar0 + 296 + 8 * a; };
     auto pfull_bar = [&](int b) { return bar0 + 320 + 8 * b; };
-    auto pempty_bar = [&](int b) { return bar0 + 336 + 8 * b; };
-    uint32_t *tmem_slot = (uint32_t *)(smem + kTcOffBar + 360);
-    volatile int *abort_flag = (volatile int *)(smem + kTcOffBar + 368);
+    auto pempty_bar = [&](int b) { return bar0 + 344 + 8 * b; };
+    uint32_t *tmem_slot = (uint32_t *)(smem + kTcOffBar + 376);
+    volatile int *abort_flag = (volatile int *)(smem + kTcOffBar + 384);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -272,7 +274,7 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
             mbar_init(afull_bar(a), 4);
             mbar_init(aempty_bar(a), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kTcPBufs; ++b) {
             mbar_init(pfull_bar(b), 1);
             mbar_init(pempty_bar(b), 8);
         }
@@ -362,21 +364,21 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                     const int N = (min(kTcMaxN, cnt - n0) + 15) & ~15;
                     const uint32_t idesc = idesc_bf16_m128(N);
                     for (int G = 0; G < p.ng; ++G, ++it) {
-                        const int xs = it % kTcXStages, as = it % kTcAStages, b = it & 1;
+                        const int xs = it % kTcXStages, as = it % kTcAStages, b = it % kTcPBufs;
                         if (lane == 0)
                             ok = mbar_wait(xfull_bar(xs), (it / kTcXStages) & 1, abort_flag, p.status) &&
                                  mbar_wait(afull_bar(as), (it / kTcAStages) & 1, abort_flag, p.status) &&
-                                 mbar_wait(pempty_bar(b), ((it >> 1) & 1) ^ 1, abort_flag, p.status);
+                                 mbar_wait(pempty_bar(b), ((it / kTcPBufs) & 1) ^ 1, abort_flag, p.status);
                         ok = __shfl_sync(0xffffffffu, ok, 0);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t a_addr = sb + kTcOffA + as * kTcABytes;
                         const uint32_t x_addr = sb + kTcOffX + xs * kTcXBytes;
                         const uint64_t ad = sw128_desc(a_addr), xd = sw128_desc(x_addr);
-                        tc_mma_elect<false>(tmem + b * 256, ad, xd, idesc);
-                        tc_mma_elect<true>(tmem + b * 256, ad + 2, xd + 2, idesc);
-                        tc_mma_elect<true>(tmem + b * 256, ad + 4, xd + 4, idesc);
-                        tc_mma_elect<true>(tmem + b * 256, ad + 6, xd + 6, idesc);
+                        tc_mma_elect<false>(tmem + b * kTcMaxN, ad, xd, idesc);
+                        tc_mma_elect<true>(tmem + b * kTcMaxN, ad + 2, xd + 2, idesc);
+                        tc_mma_elect<true>(tmem + b * kTcMaxN, ad + 4, xd + 4, idesc);
+                        tc_mma_elect<true>(tmem + b * kTcMaxN, ad + 6, xd + 6, idesc);
                         tc_commit_elect(pfull_bar(b));
                         tc_commit_elect(aempty_bar(as));
                         tc_commit_elect(xempty_bar(xs));
@@ -486,11 +488,11 @@ gq4_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__
                         s_cur = s_next;
                         if (G + 5 < p.ng) s_next = scales4(G + 5);
                     }
-                    const int b = it & 1;
-                    if (!(ok = mbar_wait(pfull_bar(b), (it >> 1) & 1, abort_flag, p.status))) break;
+                    const int b = it % kTcPBufs;
+                    if (!(ok = mbar_wait(pfull_bar(b), (it / kTcPBufs) & 1, abort_flag, p.status))) break;
                     tc_fence_after();
                     const uint64_t ss = splat2(sc);
-                    const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + b * 256;
+                    const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + b * kTcMaxN;
                     // chunks 2c + half of 32 columns; the first two are loaded together
                     const int col0 = 32 * half, col1 = 32 * (2 + half), col2 = 32 * (4 + half);
                     if (col0 < N) {
