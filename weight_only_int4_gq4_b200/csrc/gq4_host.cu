@@ -365,13 +365,14 @@ gq4_status launch_stream_k(const StreamMats &m, const SkinnyParams &p, int units
     auto kern = gq4_stream_kernel<MODE, NT, RW>;
     StreamArgs a{};
     a.stage_bytes = stream_stage_bytes(PAIR, BR, std::min(kStMaxCols, NT * 8));
-    const int budget = (int)kMaxSmem - stream_xch_bytes(RW, NT) - 16 - 1024;
+    if (ModeTraits<MODE>::kMoe && !p.unit_ctr) return GQ4_ERR_NULL;
+    const int budget = (int)kMaxSmem - stream_xch_bytes(PAIR, RW, NT) - 16 - 16 * kStQueue - 1024;
     a.nstages = std::min(8, budget / (a.stage_bytes + 16));
     if (a.nstages < 2) return GQ4_ERR_UNSUPPORTED;
     a.wrows = (int)m.wrows;
     a.srows = (int)m.srows;
     a.status = status;
-    const size_t smem = stream_smem_bytes(a.nstages, a.stage_bytes, RW, NT);
+    const size_t smem = stream_smem_bytes(a.nstages, a.stage_bytes, PAIR, RW, NT);
     if (smem > kMaxSmem) return GQ4_ERR_UNSUPPORTED;
     CUtensorMap tm[4];
     const uint64_t rows_w = (uint64_t)(m.n_experts - 1) * m.wrows + p.O;
@@ -419,13 +420,14 @@ gq4_status launch_stream_nt(const StreamMats &m, const SkinnyParams &p, int mats
                             cudaStream_t st) {
     auto units = [&](int br) { return mats * ((p.O + br - 1) / br); };
     const int want = 2 * sm_count();
-    if constexpr (ModeTraits<MODE>::kPair == 2) {
-        if (ModeTraits<MODE>::kMoe || units(128) >= want)
-            return launch_stream_k<MODE, NT, 8>(m, p, units(128), status, st);
+    if constexpr (ModeTraits<MODE>::kMoe) {
+        return launch_stream_k<MODE, NT, ModeTraits<MODE>::kPair == 2 ? 8 : 16>(m, p, units(ModeTraits<MODE>::kPair == 2 ? 128 : 256),
+                                                                                 status, st);
+    } else if constexpr (ModeTraits<MODE>::kPair == 2) {
+        if (units(128) >= want) return launch_stream_k<MODE, NT, 8>(m, p, units(128), status, st);
         return launch_stream_k<MODE, NT, 4>(m, p, units(64), status, st);
     } else {
-        if (ModeTraits<MODE>::kMoe || units(256) >= want)
-            return launch_stream_k<MODE, NT, 16>(m, p, units(256), status, st);
+        if (units(256) >= want) return launch_stream_k<MODE, NT, 16>(m, p, units(256), status, st);
         if (units(128) >= want) return launch_stream_k<MODE, NT, 8>(m, p, units(128), status, st);
         return launch_stream_k<MODE, NT, 4>(m, p, units(64), status, st);
     }
@@ -433,13 +435,20 @@ gq4_status launch_stream_nt(const StreamMats &m, const SkinnyParams &p, int mats
 
 // At most three n-tiles (24 columns) per pass: the four-tile variant needs more registers
 // than the 16 consumer warps have and spills; a matrix with more columns takes passes.
+// Routed experts take at most two (16 columns): the smaller stage leaves room for a fifth
+// ring stage, which gained more than the second pass of the few experts with 17-24 rows
+// cost (32-token decode, 64 or 32 experts: 4-8 % less time).
 template <int MODE>
 gq4_status launch_stream(const StreamMats &m, const SkinnyParams &p, int max_cols, int mats, int32_t *status,
                          cudaStream_t st) {
     const int c = std::min(max_cols, kStMaxCols);
     if (c <= 8) return launch_stream_nt<MODE, 1>(m, p, mats, status, st);
-    if (c <= 16) return launch_stream_nt<MODE, 2>(m, p, mats, status, st);
-    return launch_stream_nt<MODE, 3>(m, p, mats, status, st);
+    if constexpr (ModeTraits<MODE>::kMoe) {
+        return launch_stream_nt<MODE, 2>(m, p, mats, status, st);
+    } else {
+        if (c <= 16) return launch_stream_nt<MODE, 2>(m, p, mats, status, st);
+        return launch_stream_nt<MODE, 3>(m, p, mats, status, st);
+    }
 }
 
 template <int MODE>
@@ -845,6 +854,9 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     const int small_cols = (int)std::min<int64_t>(max_cols, tc ? kLargeMin - 1 : max_cols);
     const bool band = small_cols >= kBandMinCols;
     int32_t *status = at<int32_t>(ws, L.status);
+    // words 1 and 2 of the status block (cleared with it by the router or a memset) count
+    // the units the two decode kernels have taken
+    pg.unit_ctr = status + 1;
     const bool stream_gu = stream_usable(Wg) && stream_usable(Wu) && Wu->expert_stride_s == Wg->expert_stride_s;
     if (stream_gu)
         st = launch_stream<kMoeGateUp>(stream_mats(Wg, Wu), pg, small_cols, max_active, status, s);
@@ -902,6 +914,7 @@ gq4_status moe_expert_ffn(const gq4_tensor *Wg, const gq4_tensor *Wu, const gq4_
     pd.row_tiles = (int)((H + 15) / 16);
     pd.x = at<void>(ws, L.h); pd.xdt = 1; pd.n_tok = (int)T;
     pd.y = y;
+    pd.unit_ctr = status + 2;
     set_extents(pd, Wd, nullptr, T * K, E);
     if (stream_usable(Wd))
         st = launch_stream<kMoeDown>(stream_mats(Wd, nullptr), pd, small_cols, max_active, status, s);

@@ -166,18 +166,48 @@ __device__ __forceinline__ int block_excl_scan_1024(int v, int *sh /*[32]*/, int
 }
 
 // Expert lists for the two GEMM regimes: small (0 < cnt < thr: the decode kernels) and
-// large (cnt >= thr: the tensor-core kernels), each ascending.  Null pointers: skipped.
+// large (cnt >= thr: the tensor-core kernels).  The large list is ascending.  The small
+// list is ordered by row count, most rows first (counts from 63 up share one place; the
+// order among equal counts is not fixed): the decode kernels take their work in list
+// order, so the units that cost most start first.  Null pointers: skipped.
 struct ExpertLists {
     int32_t *n_small, *small, *n_large, *large;
     int thr;
 };
 
+constexpr int kCountBins = 64;
+
+// Called by all 1024 threads of the block; thread e = expert e with c rows.
 __device__ __forceinline__ void classify_experts(int e, int E, int c, int *sh, const ExpertLists &L) {
-    int tot;
+    __shared__ int bin_cnt[kCountBins], bin_base[kCountBins];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool is_small = e < E && c > 0 && c < L.thr, is_large = e < E && c >= L.thr;
-    const int sb = block_excl_scan_1024(is_small ? 1 : 0, sh, &tot);
-    if (is_small && L.small) L.small[sb] = e;
-    if (e == 0 && L.n_small) *L.n_small = tot;
+    // bin 0 holds the most rows
+    const int b = is_small ? kCountBins - 1 - min(c, kCountBins - 1) : -1;
+    if (threadIdx.x < kCountBins) bin_cnt[threadIdx.x] = 0;
+    __syncthreads();
+    if (b >= 0) atomicAdd(&bin_cnt[b], 1);
+    __syncthreads();
+    if (warp == 0) {  // exclusive prefix of the bin counts, in bin order
+        const int t0 = bin_cnt[lane], t1 = bin_cnt[lane + 32];
+        int x0 = t0, x1 = t1;
+        #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
+            if (lane >= o) { x0 += y0; x1 += y1; }
+        }
+        const int total0 = __shfl_sync(0xffffffffu, x0, 31);
+        bin_base[lane] = x0 - t0;
+        bin_base[lane + 32] = total0 + x1 - t1;
+        if (lane == 31 && L.n_small) *L.n_small = total0 + x1;
+    }
+    __syncthreads();
+    if (b >= 0 && L.small) L.small[atomicAdd(&bin_base[b], 1)] = e;
+    if (L.thr >= (1 << 30)) {  // no expert can reach the threshold
+        if (e == 0 && L.n_large) *L.n_large = 0;
+        return;
+    }
+    int tot;
     const int lb = block_excl_scan_1024(is_large ? 1 : 0, sh, &tot);
     if (is_large && L.large) L.large[lb] = e;
     if (e == 0 && L.n_large) *L.n_large = tot;

@@ -67,6 +67,9 @@ struct SkinnyParams {
     // floats of the scale array, rows of the activation array, experts of the call
     int64_t w_bytes, s_count, x_rows;
     int n_exp;
+    // TMA-fed decode kernel, MoE modes: device counter of the (expert, band) units taken,
+    // zero before the launch
+    int32_t *unit_ctr;
 };
 
 template <int MODE>

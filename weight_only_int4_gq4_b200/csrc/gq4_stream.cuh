@@ -15,15 +15,25 @@
 //    16 B, one TMA copy) and the stage's 256 activations of every column (one bulk copy
 //    per column; the source address does the token gather).  Completion is an mbarrier
 //    with a transaction count; no thread spends instructions on weight addresses.
-//  * Sixteen consumer warps: RW row warps x KW = 16/RW k-warps.  A row warp owns 16 rows;
-//    its k-warps split the stage's (matrix, group) items (gate+up: one matrix each; down:
-//    256-row bands need no split).  Each item is one m16n8k16 tensor op chain per 8
+//  * Sixteen consumer warps: row warps x k-warps.  The 16 accumulator rows of a warp's
+//    m16n8k16 tensor ops are 16 band rows of one matrix, or, for gate+up, 8 band rows of
+//    the gate matrix and the same 8 rows of the up matrix, so that one thread holds
+//    gate and up of the same outputs and the SiLU product needs no exchange.  When the
+//    band has fewer rows than the warps cover, k-warps split the stage's groups.  Each
+//    item (16 accumulator rows x one 64-wide group) is one tensor op chain per 8
 //    columns: the nibbles become exact bf16 integers (one lop3 + one bf16x2 fma per two
-//    weights), the f32 partial of the group is scaled by s[o][g] and added to the running
-//    sum.  The integer pipe is the scarce one (the nibble decode lives there), so every
-//    address, slot and phase is computed incrementally or once per warp.
-//  * At the end of a band the k-warps' sums are added in a fixed order through shared
-//    memory (deterministic) and the mode's epilogue runs.
+//    weights), the f32 partial of the group is scaled by its row's s[o][g] and added to
+//    the running sum.  The integer pipe is the scarce one (the nibble decode lives there),
+//    so every address, slot and phase is computed incrementally or once per warp.
+//  * With k-warps, their sums are added at the end of a band in a fixed order through
+//    shared memory (deterministic); then the mode's epilogue runs.
+//  * Routed experts (MoE modes): the (expert, band) units are taken from a counter in the
+//    order of the expert list, which the row map sorts by rows per expert, most first, so
+//    the costliest units start first and the CTAs finish together.  The producer passes
+//    each pass's band, column offset, column count and first row to the consumers in a
+//    small shared-memory queue beside the ring; a band of -1 ends the kernel.  The
+//    down projection's token indices and routing weights are read at the start of a
+//    pass, one column per lane, so their latency hides behind the pass's stages.
 // Every wait is bounded (~2 s): on expiry GQ4_ERR_TIMEOUT is raised in the status word,
 // the other waits return at once, all warps still pass the same barriers, and the
 // producer lets its copies in flight land before the CTA leaves.
@@ -41,6 +51,7 @@ constexpr int kStThreads = (kStConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kStMaxCols = 32;                            // columns per pass
 constexpr int kStXStride = 528;  // bytes per staged activation row: 256 bf16 + 16 B pad
 constexpr int kStGroups = 4;     // groups per stage (128 packed bytes per row)
+constexpr int kStQueue = 9;      // pass queue entries: ring depth (<= 8) + 1
 
 struct StreamArgs {
     int nstages;       // ring depth
@@ -50,16 +61,27 @@ struct StreamArgs {
     int32_t *status;   // device status word (GQ4_ERR_TIMEOUT), may be NULL
 };
 
+// Warp split of a band of 16*RW rows (of each matrix) over the 16 consumer warps.
+template <int PAIR, int RW>
+struct StreamSplit {
+    static constexpr int kRowsPerWarp = 16 / PAIR;            // band rows per row warp
+    static constexpr int kRowWarps = RW * PAIR;               // 16*RW / kRowsPerWarp
+    static constexpr int kKWarps = kStConsumerWarps / kRowWarps;
+    static constexpr int kGroupsPerWarp = kStGroups / kKWarps;  // per stage
+};
+
 __host__ __device__ inline int stream_stage_bytes(int pair, int br, int ncols) {
     const int b = pair * br * 128 + pair * br * 16 + ncols * kStXStride;
     return (b + 1023) & ~1023;
 }
-__host__ __device__ inline int stream_xch_bytes(int rw, int nt) {
-    return rw * (kStConsumerWarps / rw - 1) * nt * 4 * 32 * 4;
+__host__ __device__ inline int stream_xch_bytes(int pair, int rw, int nt) {
+    const int row_warps = rw * pair;
+    return row_warps * (kStConsumerWarps / row_warps - 1) * nt * 4 * 32 * 4;
 }
-// ring + exchange buffer + 2 mbarriers per stage + abort flag + 1024 for alignment
-__host__ __device__ inline int stream_smem_bytes(int nstages, int stage_bytes, int rw, int nt) {
-    return nstages * stage_bytes + stream_xch_bytes(rw, nt) + 16 * nstages + 16 + 1024;
+// ring + exchange buffer + 2 mbarriers per stage + abort flag + pass queue + 1024 for
+// alignment
+__host__ __device__ inline int stream_smem_bytes(int nstages, int stage_bytes, int pair, int rw, int nt) {
+    return nstages * stage_bytes + stream_xch_bytes(pair, rw, nt) + 16 * nstages + 16 + 16 * kStQueue + 1024;
 }
 
 // Four bf16x2 pairs of one device word (nibble slots i and i+4 -> columns 2i, 2i+1).
@@ -93,21 +115,22 @@ __device__ __forceinline__ void named_bar_consumers() {
     asm volatile("bar.sync 1, %0;" ::"r"(kStConsumerWarps * 32) : "memory");
 }
 
-// The items of one stage for one consumer warp: groups GL0 .. GL0+IPW-1 of its matrix.
-//   a_row: its packed tile row R (and R+8 at +1024); s_row: the four scales of row R (row
-//   R+8 at +128); x_lane: the activation bytes this lane feeds for n-tile 0, group 0.
+// The items of one stage for one consumer warp: groups GL0 .. GL0+IPW-1.
+//   a_row: the packed tile row of accumulator rows 0-7 (this lane: row g), A1 bytes on
+//   the tile row of rows 8-15; s_row: the four scales of the first, S1 bytes on those of
+//   the second; x_lane: the activation bytes this lane feeds for n-tile 0, group 0.
 // Columns past nc hold stale values: they only reach accumulator columns that are never
 // stored, so they need no zeroing.
-template <int NT, int NTA, int IPW, int GL0>
+template <int NT, int NTA, int IPW, int GL0, int A1, int S1>
 __device__ __forceinline__ void stream_items_n(const uint8_t *a_row, const uint8_t *s_row, const uint8_t *x_lane,
                                              const int (&aoff)[kStGroups], float (&acc)[NT][4]) {
     const float4 sva = *(const float4 *)s_row;
-    const float4 svb = *(const float4 *)(s_row + 8 * 16);
+    const float4 svb = *(const float4 *)(s_row + S1);
     #pragma unroll
     for (int q = 0; q < IPW; ++q) {
         const int gl = GL0 + q;
         const uint2 wa = *(const uint2 *)(a_row + aoff[gl]);
-        const uint2 wb = *(const uint2 *)(a_row + 8 * 128 + aoff[gl]);
+        const uint2 wb = *(const uint2 *)(a_row + A1 + aoff[gl]);
         const float sa = gl == 0 ? sva.x : gl == 1 ? sva.y : gl == 2 ? sva.z : sva.w;
         const float sb = gl == 0 ? svb.x : gl == 1 ? svb.y : gl == 2 ? svb.z : svb.w;
         const uint64_t ssa = splat2(sa), ssb = splat2(sb);
@@ -133,13 +156,13 @@ __device__ __forceinline__ void stream_items_n(const uint8_t *a_row, const uint8
     }
 }
 
-template <int NT, int IPW, int GL0>
+template <int NT, int IPW, int GL0, int A1, int S1>
 __device__ __forceinline__ void stream_items(const uint8_t *a_row, const uint8_t *s_row, const uint8_t *x_lane,
                                              const int (&aoff)[kStGroups], int nc, float (&acc)[NT][4]) {
-    if (NT >= 4 && nc > 24) stream_items_n<NT, (NT >= 4 ? 4 : 1), IPW, GL0>(a_row, s_row, x_lane, aoff, acc);
-    else if (NT >= 3 && nc > 16) stream_items_n<NT, (NT >= 3 ? 3 : 1), IPW, GL0>(a_row, s_row, x_lane, aoff, acc);
-    else if (NT >= 2 && nc > 8) stream_items_n<NT, (NT >= 2 ? 2 : 1), IPW, GL0>(a_row, s_row, x_lane, aoff, acc);
-    else stream_items_n<NT, 1, IPW, GL0>(a_row, s_row, x_lane, aoff, acc);
+    if (NT >= 4 && nc > 24) stream_items_n<NT, (NT >= 4 ? 4 : 1), IPW, GL0, A1, S1>(a_row, s_row, x_lane, aoff, acc);
+    else if (NT >= 3 && nc > 16) stream_items_n<NT, (NT >= 3 ? 3 : 1), IPW, GL0, A1, S1>(a_row, s_row, x_lane, aoff, acc);
+    else if (NT >= 2 && nc > 8) stream_items_n<NT, (NT >= 2 ? 2 : 1), IPW, GL0, A1, S1>(a_row, s_row, x_lane, aoff, acc);
+    else stream_items_n<NT, 1, IPW, GL0, A1, S1>(a_row, s_row, x_lane, aoff, acc);
 }
 
 template <int MODE, int NT, int RW>
@@ -148,25 +171,38 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
                   const __grid_constant__ CUtensorMap tm_s0, const __grid_constant__ CUtensorMap tm_s1,
                   const SkinnyParams p, const StreamArgs a) {
     using TR = ModeTraits<MODE>;
+    using SP = StreamSplit<TR::kPair, RW>;
     constexpr int PAIR = TR::kPair;
-    constexpr int BR = 16 * RW;
-    constexpr int KW = kStConsumerWarps / RW;   // k-warps per row warp
-    constexpr int IPW = kStGroups * PAIR / KW;  // (matrix, group) items per warp per stage
-    constexpr int KPM = KW / PAIR;              // k-warps per matrix
-    static_assert(IPW >= 1 && IPW <= kStGroups && KW % PAIR == 0, "item split");
+    constexpr int BR = 16 * RW;                 // band rows of each matrix
+    constexpr int RPW = SP::kRowsPerWarp;
+    constexpr int NRW = SP::kRowWarps;
+    constexpr int KW = SP::kKWarps;
+    constexpr int IPW = SP::kGroupsPerWarp;
+    static_assert(NRW * KW == kStConsumerWarps && IPW * KW == kStGroups, "warp split");
     constexpr int WBOX = BR * 128, SBOX = BR * 16;
     constexpr int XOFF = PAIR * (WBOX + SBOX);
+    // tile and scale offsets of accumulator rows 8-15: the up matrix's rows for gate+up,
+    // else band rows R+8
+    constexpr int A1 = PAIR == 2 ? WBOX : 8 * 128;
+    constexpr int S1 = PAIR == 2 ? SBOX : 8 * 16;
     constexpr int PW = NT * 8 < kStMaxCols ? NT * 8 : kStMaxCols;  // columns per pass (x rows a stage holds)
+    // routed experts take their units from a counter; the other modes walk them statically
+    constexpr bool kDyn = TR::kMoe;
+    static_assert(!kDyn || KW == 1, "a queue-fed consumer runs no exchange barrier");
 
     extern __shared__ uint8_t st_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)st_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(sm);
     const int NS = a.nstages, SB = a.stage_bytes;
+    constexpr int XCH = (NRW * (KW - 1) * NT * 4 * 32 * 4);
     float *xch = (float *)(sm + NS * SB);
-    const uint32_t bar0 = sbase + NS * SB + stream_xch_bytes(RW, NT);
+    const uint32_t bar0 = sbase + NS * SB + XCH;
     auto full_bar = [&](int s) { return bar0 + 8 * s; };
     auto empty_bar = [&](int s) { return bar0 + 8 * (NS + s); };
-    volatile int *abort_flag = (volatile int *)(sm + NS * SB + stream_xch_bytes(RW, NT) + 16 * NS);
+    volatile int *abort_flag = (volatile int *)(sm + NS * SB + XCH + 16 * NS);
+    // pass queue: {band (-1: end), first column, columns, first row}; its entries are
+    // ordered by the ring's mbarriers (the asm statements clobber memory)
+    int4 *queue = (int4 *)(sm + NS * SB + XCH + 16 * NS + 16);
     int32_t *status = a.status;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,22 +234,38 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
     const int n_units = TR::kMoe ? (*p.n_active) * bands : bands;
     const int nst = p.ng / kStGroups;  // stages per pass
 
-    uint32_t issued = 0;  // stages the producer warp issued
+    uint32_t issued = 0;  // ring entries the producer warp filled (stages and the end marker)
     if (warp == kStConsumerWarps) {
         // ------------------------------------------------------------ producer warp
-        int s = 0;
+        int s = 0, seq = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-            int e = 0, band = u, row0 = 0, cols = p.n_tok;
+        // expert, first row and columns of unit uu (routed experts: two dependent loads)
+        auto unit_info = [&](int uu, int &e, int &row0, int &cols) {
+            e = 0; row0 = 0; cols = p.n_tok;
             if (TR::kMoe) {
-                const int ai = u / bands;
-                band = u - ai * bands;
-                e = p.active[ai];
+                e = p.active[uu / bands];
                 if (!in_bounds(e, p.n_exp)) e = 0;  // the stages must still be delivered
                 row0 = p.offs[e];
                 cols = p.cnt[e];
             }
+        };
+        int u = blockIdx.x;
+        if (kDyn) {
+            int v = 0;
+            if (lane == 0) v = atomicAdd(p.unit_ctr, 1);
+            u = __shfl_sync(0xffffffffu, v, 0);
+        }
+        int e = 0, row0 = 0, cols = 0;
+        if (u < n_units) unit_info(u, e, row0, cols);
+        while (u < n_units) {
+            const int band = TR::kMoe ? u % bands : u;
+            // the next unit is claimed now and its expert read at this unit's second ring
+            // entry, so that neither latency falls between two units
+            int u_nx = u + gridDim.x, e_nx = 0, row0_nx = 0, cols_nx = 0;
+            bool have_nx = false;
+            if (kDyn && lane == 0) u_nx = atomicAdd(p.unit_ctr, 1);
+            int entry = 0;
             const int wrow = e * a.wrows + band * BR, srow = e * a.srows + band * BR;
             for (int c0 = 0; c0 < cols; c0 += PW) {
                 const int nc = min(PW, cols - c0);
@@ -227,12 +279,19 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
                     xrow = (const uint16_t *)p.x + xr * p.I;
                 }
                 const uint32_t tx = (uint32_t)(XOFF + nc * 512);
-                for (int k = 0; k < nst; ++k) {
+                for (int k = 0; k < nst; ++k, ++entry) {
+                    if (kDyn && entry == 1) {
+                        u_nx = __shfl_sync(0xffffffffu, u_nx, 0);
+                        if (u_nx < n_units) unit_info(u_nx, e_nx, row0_nx, cols_nx);
+                        have_nx = true;
+                    }
                     if (ok && lane == 0) ok = st_wait(empty_bar(s), ph ^ 1u, abort_flag, status) && !*abort_flag;
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (ok) {
                         const uint32_t stg = sbase + s * SB;
                         if (lane == 0) {
+                            // the queue entry is published by the arrive below (release)
+                            if (kDyn && k == 0) queue[seq % kStQueue] = make_int4(band, c0, nc, row0);
                             mbar_expect_tx(full_bar(s), tx);
                             tma_load_2d(stg, &tm_w0, k * 128, wrow, full_bar(s));
                             if (PAIR == 2) tma_load_2d(stg + WBOX, &tm_w1, k * 128, wrow, full_bar(s));
@@ -247,122 +306,159 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
                     }
                     if (++s == NS) { s = 0; ph ^= 1u; }
                 }
+                ++seq;
+            }
+            if (kDyn && !ok) break;  // the consumers leave at their next failed wait
+            if (kDyn) u_nx = __shfl_sync(0xffffffffu, u_nx, 0);
+            if (!have_nx && u_nx < n_units) unit_info(u_nx, e_nx, row0_nx, cols_nx);
+            u = u_nx; e = e_nx; row0 = row0_nx; cols = cols_nx;
+        }
+        if (kDyn && ok) {
+            // end marker: a ring entry with no copies whose queue entry has band -1
+            if (lane == 0) ok = st_wait(empty_bar(s), ph ^ 1u, abort_flag, status) && !*abort_flag;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok) {
+                if (lane == 0) {
+                    queue[seq % kStQueue] = make_int4(-1, 0, 0, 0);
+                    mbar_arrive(full_bar(s));
+                }
+                ++issued;
             }
         }
     } else {
         // ------------------------------------------------------------ consumer warps
         const int g = lane >> 2, t = lane & 3;
-        const int rw = warp % RW, kw = warp / RW;
-        const int m = (kw * IPW) / kStGroups;    // matrix of this warp's items
-        const int gl0 = (kw * IPW) % kStGroups;  // its first group in a stage
-        const int R = 16 * rw + g;               // band row of accumulator slots 0,1 (2,3: R+8)
+        const int rw = warp % NRW, kw = warp / NRW;
+        const int gl0 = kw * IPW;   // this warp's first group in a stage
+        const int R = RPW * rw + g; // band row of accumulator slots 0,1 (and of 2,3 for gate+up)
         // 128B swizzle: 16-byte chunk c of tile row r sits at chunk c ^ (r & 7), and
         // (R & 7) == ((R + 8) & 7) == g; lane t reads bytes 8t..8t+7 of each group
         int aoff[kStGroups];
         #pragma unroll
         for (int gl = 0; gl < kStGroups; ++gl) aoff[gl] = (((2 * gl + (t >> 1)) ^ g) << 4) | ((t & 1) << 3);
-        const int a_base = m * WBOX + R * 128;
-        const int s_base = PAIR * WBOX + m * SBOX + R * 16;
+        const int a_base = R * 128;
+        const int s_base = PAIR * WBOX + R * 16;
         const int x_base = XOFF + g * kStXStride + t * 32;
-        int s = 0;
+        int s = 0, seq = 0;
         uint32_t ph = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-            int e = 0, band = u, row0 = 0, cols = p.n_tok;
-            if (TR::kMoe) {
-                const int ai = u / bands;
-                band = u - ai * bands;
-                e = p.active[ai];
-                if (kChecked && (e < 0 || e >= p.n_exp)) e = 0;  // as the producer substituted
-                row0 = p.offs[e];
-                cols = p.cnt[e];
+        int su = blockIdx.x, sc0 = 0;  // static walk: unit and first column of the next pass
+        for (;;) {
+            int band, c0, nc, row0;
+            bool waited = false;  // the pass's first stage has been waited for
+            if constexpr (kDyn) {
+                if (!st_wait(full_bar(s), ph, abort_flag, status)) break;
+                const int4 q = queue[seq % kStQueue];
+                if (q.x < 0) break;
+                band = q.x; c0 = q.y; nc = q.z; row0 = q.w;
+                waited = true;
+            } else {
+                if (su >= n_units || p.n_tok <= 0) break;
+                band = su; c0 = sc0; row0 = 0;
+                nc = min(PW, p.n_tok - c0);
+                if (sc0 + PW < p.n_tok) sc0 += PW;
+                else { sc0 = 0; su += gridDim.x; }
             }
-            for (int c0 = 0; c0 < cols; c0 += PW) {
-                const int nc = min(PW, cols - c0);
-                float acc[NT][4];
+            // down projection: token and routing weight of column `lane` of this pass
+            int tok_l = -1;
+            float wt_l = 0.f;
+            if (MODE == kMoeDown && lane < nc) {
+                const int r = row0 + c0 + lane;
+                tok_l = p.row_tok[r];
+                wt_l = p.wts[p.row_slot[r]];
+            }
+            float acc[NT][4];
+            #pragma unroll
+            for (int n = 0; n < NT; ++n)
                 #pragma unroll
-                for (int n = 0; n < NT; ++n)
-                    #pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+                for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
 
-                for (int k = 0; k < nst; ++k) {
-                    if (st_wait(full_bar(s), ph, abort_flag, status)) {
-                        const uint8_t *stg = sm + s * SB;
-                        const uint8_t *ar = stg + a_base, *sr = stg + s_base, *xl = stg + x_base;
-                        if constexpr (IPW == 4) {
-                            stream_items<NT, 4, 0>(ar, sr, xl, aoff, nc, acc);
-                        } else if constexpr (IPW == 2) {
-                            if (gl0 == 0) stream_items<NT, 2, 0>(ar, sr, xl, aoff, nc, acc);
-                            else stream_items<NT, 2, 2>(ar, sr, xl, aoff, nc, acc);
-                        } else {
-                            if (gl0 == 0) stream_items<NT, 1, 0>(ar, sr, xl, aoff, nc, acc);
-                            else if (gl0 == 1) stream_items<NT, 1, 1>(ar, sr, xl, aoff, nc, acc);
-                            else if (gl0 == 2) stream_items<NT, 1, 2>(ar, sr, xl, aoff, nc, acc);
-                            else stream_items<NT, 1, 3>(ar, sr, xl, aoff, nc, acc);
-                        }
+            bool aborted = false;
+            for (int k = 0; k < nst; ++k) {
+                const bool have = (k == 0 && waited) || st_wait(full_bar(s), ph, abort_flag, status);
+                if (have) {
+                    const uint8_t *stg = sm + s * SB;
+                    const uint8_t *ar = stg + a_base, *sr = stg + s_base, *xl = stg + x_base;
+                    if constexpr (IPW == 4) {
+                        stream_items<NT, 4, 0, A1, S1>(ar, sr, xl, aoff, nc, acc);
+                    } else if constexpr (IPW == 2) {
+                        if (gl0 == 0) stream_items<NT, 2, 0, A1, S1>(ar, sr, xl, aoff, nc, acc);
+                        else stream_items<NT, 2, 2, A1, S1>(ar, sr, xl, aoff, nc, acc);
+                    } else {
+                        if (gl0 == 0) stream_items<NT, 1, 0, A1, S1>(ar, sr, xl, aoff, nc, acc);
+                        else if (gl0 == 1) stream_items<NT, 1, 1, A1, S1>(ar, sr, xl, aoff, nc, acc);
+                        else if (gl0 == 2) stream_items<NT, 1, 2, A1, S1>(ar, sr, xl, aoff, nc, acc);
+                        else stream_items<NT, 1, 3, A1, S1>(ar, sr, xl, aoff, nc, acc);
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(empty_bar(s));
-                    if (++s == NS) { s = 0; ph ^= 1u; }
+                } else if (kDyn) {
+                    aborted = true;  // no barrier below needs this warp: leave
+                    break;
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(s));
+                if (++s == NS) { s = 0; ph ^= 1u; }
+            }
+            if (aborted) break;
+            ++seq;
 
-                // ---- combine the k-warps (fixed order) and run the epilogue
-                float v0[NT][4], v1[NT][4];
-                if constexpr (KW > 1) {
-                    if (kw != 0) {
-                        float *dst = xch + (rw * (KW - 1) + kw - 1) * NT * 4 * 32 + lane;
+            // ---- add the k-warps' sums (fixed order) and run the epilogue
+            float v[NT][4];
+            if constexpr (KW > 1) {
+                if (kw != 0) {
+                    float *dst = xch + (rw * (KW - 1) + kw - 1) * NT * 4 * 32 + lane;
+                    #pragma unroll
+                    for (int n = 0; n < NT; ++n)
                         #pragma unroll
-                        for (int n = 0; n < NT; ++n)
-                            #pragma unroll
-                            for (int i = 0; i < 4; ++i) dst[(n * 4 + i) * 32] = acc[n][i];
-                    }
-                    named_bar_consumers();
-                    if (kw == 0) {
-                        #pragma unroll
-                        for (int n = 0; n < NT; ++n)
-                            #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                float s0 = acc[n][i], s1 = 0.f;
-                                #pragma unroll
-                                for (int w = 1; w < KW; ++w) {
-                                    const float v = xch[((rw * (KW - 1) + w - 1) * NT * 4 + n * 4 + i) * 32 + lane];
-                                    if (w < KPM) s0 += v; else s1 += v;
-                                }
-                                v0[n][i] = s0;
-                                v1[n][i] = s1;
-                            }
-                    }
-                    named_bar_consumers();  // the exchange buffer may be rewritten
-                } else {
+                        for (int i = 0; i < 4; ++i) dst[(n * 4 + i) * 32] = acc[n][i];
+                }
+                named_bar_consumers();
+                if (kw == 0) {
                     #pragma unroll
                     for (int n = 0; n < NT; ++n)
                         #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            v0[n][i] = acc[n][i];
-                            v1[n][i] = 0.f;
+                            float sum = acc[n][i];
+                            #pragma unroll
+                            for (int w = 1; w < KW; ++w)
+                                sum += xch[((rw * (KW - 1) + w - 1) * NT * 4 + n * 4 + i) * 32 + lane];
+                            v[n][i] = sum;
                         }
                 }
-                if (kw == 0 && !*abort_flag) {
+                named_bar_consumers();  // the exchange buffer may be rewritten
+            } else {
+                #pragma unroll
+                for (int n = 0; n < NT; ++n)
                     #pragma unroll
-                    for (int n = 0; n < NT; ++n) {
+                    for (int i = 0; i < 4; ++i) v[n][i] = acc[n][i];
+            }
+            if (kw == 0 && !*abort_flag) {
+                #pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    if constexpr (PAIR == 2) {
+                        // slots 0,1: gate of row R, columns 2t, 2t+1; slots 2,3: up of the same
+                        #pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const int cl = n * 8 + 2 * t + i;
+                            const int o = band * BR + R;
+                            if (cl >= nc || o >= p.O) continue;
+                            const int c = c0 + cl;
+                            const uint16_t hv = (uint16_t)bf16_bits_rn(silu_mul(v[n][i], v[n][i + 2]));
+                            if (MODE == kGateUp) ((uint16_t *)p.h)[(int64_t)c * p.O + o] = hv;
+                            else ((uint16_t *)p.h)[(int64_t)(row0 + c) * p.O + o] = hv;
+                        }
+                    } else {
                         #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const int cl = n * 8 + 2 * t + (i & 1);
                             const int o = band * BR + R + ((i >> 1) << 3);
-                            if (cl >= nc || o >= p.O) continue;
-                            const int c = c0 + cl;
-                            if (MODE == kMatvec) {
-                                p.y[(int64_t)c * p.O + o] = v0[n][i];
-                            } else if (MODE == kGateUp) {
-                                ((uint16_t *)p.h)[(int64_t)c * p.O + o] =
-                                    (uint16_t)bf16_bits_rn(silu_mul(v0[n][i], v1[n][i]));
-                            } else if (MODE == kMoeGateUp) {
-                                ((uint16_t *)p.h)[(int64_t)(row0 + c) * p.O + o] =
-                                    (uint16_t)bf16_bits_rn(silu_mul(v0[n][i], v1[n][i]));
+                            if (MODE == kMoeDown) {
+                                // every lane takes part in the shuffles
+                                const int tok = __shfl_sync(0xffffffffu, tok_l, cl & 31);
+                                const float wt = __shfl_sync(0xffffffffu, wt_l, cl & 31);
+                                if (cl >= nc || o >= p.O) continue;
+                                if (in_bounds(tok, p.n_tok)) atomicAdd(p.y + (int64_t)tok * p.O + o, wt * v[n][i]);
                             } else {
-                                const int r = row0 + c;
-                                const int tok = p.row_tok[r];
-                                if (in_bounds(tok, p.n_tok))
-                                    atomicAdd(p.y + (int64_t)tok * p.O + o, p.wts[p.row_slot[r]] * v0[n][i]);
+                                if (cl >= nc || o >= p.O) continue;
+                                p.y[(int64_t)(c0 + cl) * p.O + o] = v[n][i];
                             }
                         }
                     }
