@@ -34,9 +34,11 @@
 //    small shared-memory queue beside the ring; a band of -1 ends the kernel.  The
 //    down projection's token indices and routing weights are read at the start of a
 //    pass, one column per lane, so their latency hides behind the pass's stages.
-// Every wait is bounded (~2 s): on expiry GQ4_ERR_TIMEOUT is raised in the status word,
-// the other waits return at once, all warps still pass the same barriers, and the
-// producer lets its copies in flight land before the CTA leaves.
+// Every wait is bounded (~2 s): on expiry GQ4_ERR_TIMEOUT is raised in the status word
+// and the other waits return at once.  Warps that share a barrier (the k-warps of the
+// dense modes) still pass it; the queue-fed consumers of routed experts, which share
+// none, leave at their next failed wait.  The producer lets its copies in flight land
+// before the CTA leaves.
 #pragma once
 #include <cuda.h>
 
