@@ -42,6 +42,8 @@
 #pragma once
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "gq4_common.cuh"
 #include "gq4_skinny.cuh"
 #include "gq4_tc.cuh"
@@ -156,15 +158,6 @@ __device__ __forceinline__ void stream_items_n(const uint8_t *a_row, const uint8
             fma2(acc[n][2], acc[n][3], d[2], d[3], ssb);
         }
     }
-}
-
-template <int NT, int IPW, int GL0, int A1, int S1>
-__device__ __forceinline__ void stream_items(const uint8_t *a_row, const uint8_t *s_row, const uint8_t *x_lane,
-                                             const int (&aoff)[kStGroups], int nc, float (&acc)[NT][4]) {
-    if (NT >= 4 && nc > 24) stream_items_n<NT, (NT >= 4 ? 4 : 1), IPW, GL0, A1, S1>(a_row, s_row, x_lane, aoff, acc);
-    else if (NT >= 3 && nc > 16) stream_items_n<NT, (NT >= 3 ? 3 : 1), IPW, GL0, A1, S1>(a_row, s_row, x_lane, aoff, acc);
-    else if (NT >= 2 && nc > 8) stream_items_n<NT, (NT >= 2 ? 2 : 1), IPW, GL0, A1, S1>(a_row, s_row, x_lane, aoff, acc);
-    else stream_items_n<NT, 1, IPW, GL0, A1, S1>(a_row, s_row, x_lane, aoff, acc);
 }
 
 template <int MODE, int NT, int RW>
@@ -375,30 +368,37 @@ gq4_stream_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_consta
                 for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
 
             bool aborted = false;
-            for (int k = 0; k < nst; ++k) {
-                const bool have = (k == 0 && waited) || st_wait(full_bar(s), ph, abort_flag, status);
-                if (have) {
-                    const uint8_t *stg = sm + s * SB;
-                    const uint8_t *ar = stg + a_base, *sr = stg + s_base, *xl = stg + x_base;
-                    if constexpr (IPW == 4) {
-                        stream_items<NT, 4, 0, A1, S1>(ar, sr, xl, aoff, nc, acc);
-                    } else if constexpr (IPW == 2) {
-                        if (gl0 == 0) stream_items<NT, 2, 0, A1, S1>(ar, sr, xl, aoff, nc, acc);
-                        else stream_items<NT, 2, 2, A1, S1>(ar, sr, xl, aoff, nc, acc);
-                    } else {
-                        if (gl0 == 0) stream_items<NT, 1, 0, A1, S1>(ar, sr, xl, aoff, nc, acc);
-                        else if (gl0 == 1) stream_items<NT, 1, 1, A1, S1>(ar, sr, xl, aoff, nc, acc);
-                        else if (gl0 == 2) stream_items<NT, 1, 2, A1, S1>(ar, sr, xl, aoff, nc, acc);
-                        else stream_items<NT, 1, 3, A1, S1>(ar, sr, xl, aoff, nc, acc);
+            // the pass's stages with the active n-tile count fixed for the whole pass
+            auto run_pass = [&](auto nta_c) {
+                constexpr int NTA = decltype(nta_c)::value;
+                for (int k = 0; k < nst; ++k) {
+                    const bool have = (k == 0 && waited) || st_wait(full_bar(s), ph, abort_flag, status);
+                    if (have) {
+                        const uint8_t *stg = sm + s * SB;
+                        const uint8_t *ar = stg + a_base, *sr = stg + s_base, *xl = stg + x_base;
+                        if constexpr (IPW == 4) {
+                            stream_items_n<NT, NTA, 4, 0, A1, S1>(ar, sr, xl, aoff, acc);
+                        } else if constexpr (IPW == 2) {
+                            if (gl0 == 0) stream_items_n<NT, NTA, 2, 0, A1, S1>(ar, sr, xl, aoff, acc);
+                            else stream_items_n<NT, NTA, 2, 2, A1, S1>(ar, sr, xl, aoff, acc);
+                        } else {
+                            if (gl0 == 0) stream_items_n<NT, NTA, 1, 0, A1, S1>(ar, sr, xl, aoff, acc);
+                            else if (gl0 == 1) stream_items_n<NT, NTA, 1, 1, A1, S1>(ar, sr, xl, aoff, acc);
+                            else if (gl0 == 2) stream_items_n<NT, NTA, 1, 2, A1, S1>(ar, sr, xl, aoff, acc);
+                            else stream_items_n<NT, NTA, 1, 3, A1, S1>(ar, sr, xl, aoff, acc);
+                        }
+                    } else if (kDyn) {
+                        aborted = true;  // no barrier below needs this warp: leave
+                        break;
                     }
-                } else if (kDyn) {
-                    aborted = true;  // no barrier below needs this warp: leave
-                    break;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty_bar(s));
+                    if (++s == NS) { s = 0; ph ^= 1u; }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
-                if (++s == NS) { s = 0; ph ^= 1u; }
-            }
+            };
+            if (NT >= 3 && nc > 16) run_pass(std::integral_constant<int, (NT >= 3 ? 3 : 1)>{});
+            else if (NT >= 2 && nc > 8) run_pass(std::integral_constant<int, (NT >= 2 ? 2 : 1)>{});
+            else run_pass(std::integral_constant<int, 1>{});
             if (aborted) break;
             ++seq;
 
